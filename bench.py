@@ -1,0 +1,390 @@
+#!/usr/bin/env python
+"""Benchmark of absorbed-MLA decode on B200: one JSON line on rank 0.
+
+Workload: paged absorbed decode, B=64 sequences x H=128 heads, every sequence
+T=8192 tokens (64-token pages, shuffled block table, latent dims ~N(0, 0.25),
+rope dims and q ~N(0,1), bf16), softmax scale 1/sqrt(192), seed 3.  A step is
+one mla_decode call: the split schedule, the split-KV decode kernel and the LSE
+combine.  The 630 MB working set is larger than the 126 MB L2, so consecutive
+steps stream the cache from HBM.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+With N > 1 it runs under torchrun, one replica per GPU (no data-path
+collective; the process group only times the job as the max over ranks).
+``--impl reference`` times the fp64 CPU oracle on the host cores instead.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "MLA decode µs/step, KV HBM TB/s & % roofline at B=64,H=128,T=8192"
+UNIT = "us/step"
+B, H, T, PAGE, D, DV = 64, 128, 8192, 64, 576, 512
+SEED = 3
+WORKLOAD = ("paged absorbed MLA decode, B=64 seqs x H=128 heads, T=8192 tokens each, 576-wide bf16 rows "
+            "(512 latent x0.5 + 64 rope), 64-token pages, shuffled block table, softmax_scale=1/sqrt(192), seed 3")
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+
+
+def algorithmic_bytes(b: int, h: int, t: int, max_blocks: int) -> int:
+    """Bytes a decode step must move at least once: every cached row (576 bf16),
+    q' (576 bf16 per head), out (512 fp32 per head), lse, block table, lengths."""
+    per_seq = h * D * 2 + h * DV * 4 + h * 4 + max_blocks * 4 + 4
+    return b * t * D * 2 + b * per_seq
+
+
+def algorithmic_flops(b: int, h: int, t: int) -> int:
+    """2 flops per multiply-add: scores over 576 dims and values over 512 dims."""
+    return 2 * b * h * t * (D + DV)
+
+
+def measured_peaks() -> tuple[dict, str]:
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            return json.load(f), "measured"
+    return {"hbm_gbs": FALLBACK_HBM_GBS, "bf16_tflops": FALLBACK_BF16_TFLOPS}, "fallback"
+
+
+def decode_source_hash() -> str:
+    """Hash of the decode kernels' sources, to tie an ncu traffic figure to them."""
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "mla_latent_kv_22_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        if name.startswith("decode") or name in ("mla_device.cuh", "combine.cu", "schedule.cu"):
+            with open(os.path.join(csrc, name), "rb") as f:
+                h.update(name.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(kernel_hash: str):
+    """DRAM bytes per decode launch from the committed ncu summary, if it was taken
+    on the current sources (else None)."""
+    p = os.path.join(ROOT, "profiles", "decode_headline_traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    if d.get("source_hash") != kernel_hash:
+        return None
+    return d.get("dram_bytes_per_launch")
+
+
+# ---------------------------------------------------------------------------
+# Distributed plumbing (replicas only: barrier + max over ranks).
+# ---------------------------------------------------------------------------
+
+def dist_env() -> tuple[int, int, int]:
+    return int(os.environ.get("RANK", 0)), int(os.environ.get("LOCAL_RANK", 0)), int(os.environ.get("WORLD_SIZE", 1))
+
+
+def init_dist(backend: str):
+    import torch.distributed as dist
+    rank, _, world = dist_env()
+    if world > 1 and not dist.is_initialized():
+        dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=120))
+    return dist if world > 1 else None
+
+
+def max_over_ranks(value: float, dist, device=None) -> float:
+    if dist is None:
+        return value
+    import torch
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(dist, device=None) -> None:
+    if dist is not None:
+        if device is not None and device.type == "cuda":
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+
+
+# ---------------------------------------------------------------------------
+# Clocks during the timed region (NVML polling thread).
+# ---------------------------------------------------------------------------
+
+_REASONS = {
+    0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
+    0x10: "sync_boost", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+    0x100: "display_clock_setting",
+}
+
+
+class ClockSampler:
+    def __init__(self, device_index: int):
+        self.samples: list[tuple[int, int, int]] = []
+        self._stop = threading.Event()
+        self._ok = False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+            self._ok = True
+        except Exception as e:  # no NVML: report that
+            self.error = str(e)
+            self.max_mhz = None
+
+    def _run(self):
+        nv = self._nv
+        while not self._stop.is_set():
+            try:
+                sm = nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM)
+                rs = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                util = nv.nvmlDeviceGetUtilizationRates(self._h).gpu
+                self.samples.append((sm, rs, util))
+            except Exception:
+                pass
+            time.sleep(0.002)
+
+    def __enter__(self):
+        if self._ok:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *exc):
+        if self._ok:
+            self._stop.set()
+            self._t.join()
+
+    def summary(self) -> dict:
+        if not self._ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0, "error": getattr(self, "error", "")}
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0}
+        mhz = [s[0] for s in self.samples]
+        mask = 0
+        for s in self.samples:
+            mask |= s[1]
+        reasons = [n for bit, n in _REASONS.items() if mask & bit and n != "gpu_idle"]
+        return {"sm_mhz": statistics.median(mhz), "sm_max_mhz": self.max_mhz, "reasons": reasons,
+                "samples": len(self.samples), "sm_mhz_min": min(mhz)}
+
+
+# ---------------------------------------------------------------------------
+# CPU baseline: the fp64 oracle on a bounded sample of the workload.
+# ---------------------------------------------------------------------------
+
+def oracle_case_sample(n_seq: int):
+    import mla_synth as S
+    return S.make_decode_case(n_seq, H, T, seed=SEED, poison=False, latent_std=0.5, rope_std=1.0)
+
+
+def blas_threads() -> int:
+    try:
+        import threadpoolctl
+        info = threadpoolctl.threadpool_info()
+        return max([i.get("num_threads", 1) for i in info if i.get("user_api") == "blas"] or [1])
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def time_oracle_step(case) -> float:
+    """Seconds the oracle takes for all heads of the sample's sequences."""
+    import oracle as O
+    t0 = time.perf_counter()
+    O.mla_decode_ref(case.q, case.kv_cache, case.block_table, case.cache_seqlens, case.softmax_scale)
+    return time.perf_counter() - t0
+
+
+def cpu_baseline(budget_s: float = 15.0) -> dict:
+    case = oracle_case_sample(1)
+    t1 = time_oracle_step(case)  # one sequence, all 128 heads
+    reps = max(1, min(64, int(budget_s / max(t1, 1e-3))))
+    ts = [time_oracle_step(case) for _ in range(reps)]
+    per_seq = statistics.median(ts)
+    return {"value": per_seq * B * 1e6, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+            "sample": f"fp64 numpy oracle on 1 of the 64 sequences (all 128 heads, T=8192), median of {reps} runs, "
+                      f"scaled x64 to the full step"}
+
+
+def run_reference(args) -> None:
+    rank, _, world = dist_env()
+    if world > 1 and rank != 0:
+        return
+    case = oracle_case_sample(1)
+    for _ in range(args.warmup):
+        time_oracle_step(case)
+    ts = [time_oracle_step(case) for _ in range(args.steps)]
+    us = statistics.mean(ts) * B * 1e6
+    line = {
+        "impl": "reference", "metric": METRIC, "value": us, "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": us / 1e3, "higher_is_better": False, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "global_batch": B, "seq_len": T, "heads": H,
+                   "sample": "each step: 1 of 64 sequences, all heads; value scaled x64"},
+        "cpu_baseline": {"value": us, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+                         "sample": "each step times the fp64 oracle on 1 of the 64 sequences, scaled x64"},
+        "e2e": {"value": us, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------------------
+# Our arm.
+# ---------------------------------------------------------------------------
+
+def run_ours(args) -> None:
+    import torch
+
+    import mla_latent_kv_22_b200 as M
+    import mla_synth as S
+
+    rank, local_rank, world = dist_env()
+    torch.cuda.set_device(local_rank)
+    device = torch.device("cuda", local_rank)
+    dist = init_dist("nccl")
+
+    case = S.config_case(3, headline=True, poison=False)
+    to_dev = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(device)
+    q, kv = to_dev(case.q), to_dev(case.kv_cache)
+    bt = torch.from_numpy(case.block_table).to(device)
+    sl = torch.from_numpy(case.cache_seqlens).to(device)
+    out = torch.empty(B, H, DV, device=device)
+    lse = torch.empty(B, H, device=device)
+    max_blocks = int(case.block_table.shape[1])
+    stream = torch.cuda.current_stream(device)
+
+    def step():
+        M.mla_decode(q, kv, bt, sl, out, lse, case.softmax_scale, stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(device)
+    if M.mla_get_device_error() != 0:
+        raise RuntimeError("device error during warm-up")
+
+    # ---- device-timed region: exactly K steps ----
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    M.mla_timing_enable(True)
+    barrier(dist, device)
+    torch.cuda.synchronize(device)
+    with ClockSampler(local_rank) as clk:
+        e0.record(stream)
+        for _ in range(args.steps):
+            step()
+        e1.record(stream)
+        torch.cuda.synchronize(device)
+    barrier(dist, device)
+    ms_total = e0.elapsed_time(e1)
+    kern_ms, calls = M.mla_timing_read()
+    M.mla_timing_enable(False)
+    ms_step = max_over_ranks(ms_total / args.steps, dist, device)
+    if M.mla_get_device_error() != 0:
+        raise RuntimeError("device error during the timed region")
+
+    # ---- end to end through the public API: host buffers, copies inside the region ----
+    q_h = torch.from_numpy(np.ascontiguousarray(case.q).view(np.int16)).view(torch.bfloat16).pin_memory()
+    bt_h = torch.from_numpy(case.block_table).pin_memory()
+    sl_h = torch.from_numpy(case.cache_seqlens).pin_memory()
+    out_h = torch.empty(B, H, DV).pin_memory()
+    lse_h = torch.empty(B, H).pin_memory()
+    q_d, bt_d, sl_d = torch.empty_like(q), torch.empty_like(bt), torch.empty_like(sl)
+
+    def e2e_step():
+        q_d.copy_(q_h, non_blocking=True)
+        bt_d.copy_(bt_h, non_blocking=True)
+        sl_d.copy_(sl_h, non_blocking=True)
+        M.mla_decode(q_d, kv, bt_d, sl_d, out, lse, case.softmax_scale, stream=stream)
+        out_h.copy_(out, non_blocking=True)
+        lse_h.copy_(lse, non_blocking=True)
+
+    for _ in range(max(3, args.warmup)):
+        e2e_step()
+    torch.cuda.synchronize(device)
+    barrier(dist, device)
+    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    f0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    f1.record(stream)
+    torch.cuda.synchronize(device)
+    barrier(dist, device)
+    e2e_ms = max_over_ranks(f0.elapsed_time(f1) / args.steps, dist, device)
+    h2d = q_h.numel() * 2 + bt_h.numel() * 4 + sl_h.numel() * 4
+    d2h = out_h.numel() * 4 + lse_h.numel() * 4
+
+    if rank != 0:
+        if dist is not None:
+            dist.destroy_process_group()
+        return
+
+    peaks, peak_kind = measured_peaks()
+    alg_bytes = algorithmic_bytes(B, H, T, max_blocks)
+    flops = algorithmic_flops(B, H, T)
+    dec_ms = kern_ms[1] / max(calls, 1)
+    achieved = alg_bytes / (dec_ms * 1e-3) / 1e9  # GB/s
+    hbm_peak = float(peaks["hbm_gbs"])
+    roofline_us = max(alg_bytes / (hbm_peak * 1e9), flops / (float(peaks["bf16_tflops"]) * 1e12)) * 1e6
+    khash = decode_source_hash()
+    traffic = ncu_traffic(khash)
+    us_step = ms_step * 1e3
+    line = {
+        "metric": METRIC, "value": us_step, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": False, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "global_batch": B * world, "seq_len": T, "heads": H, "page": PAGE,
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                   "l2": "inputs larger than L2 (630 MB working set, 126 MB L2); no flush"},
+        "kv_tbps": B * T * D * 2 / (ms_step * 1e-3) / 1e12,
+        "tflops": flops / (ms_step * 1e-3) / 1e12,
+        "roofline_us": roofline_us,
+        "step_roofline_frac": roofline_us / us_step,
+        "launch_us": {"schedule": kern_ms[0] / max(calls, 1) * 1e3, "decode": dec_ms * 1e3,
+                      "combine": kern_ms[2] / max(calls, 1) * 1e3},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
+                     "frac": achieved / hbm_peak, "traffic": traffic,
+                     "peak_kind": peak_kind, "kernel": "decode (split-KV)",
+                     "algorithmic_bytes_per_launch": alg_bytes, "source_hash": khash},
+        "gpu_launches": 3 * args.steps,
+        "e2e": {"value": e2e_ms * 1e3, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "clocks": clk.summary(),
+        "decode_kernel": {0: "auto", 1: "mma.sync", 2: "tcgen05"}[M.mla_get_knob("decode_kernel")],
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline()
+    print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.destroy_process_group()
+
+
+def main() -> None:
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,338 @@
+// C ABI of libmla.so (declared in include/mla.h): argument checks, per-device
+// state (workspace, error word, SM count), and the launch sequence of each call.
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <atomic>
+#include <cstdarg>
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include "mla.h"
+#include "mla_internal.h"
+
+namespace mla {
+// Defined in decode_tc.cu.
+cudaError_t launch_decode_tc(const DecodeArgs& a, cudaStream_t stream);
+bool decode_tc_supported(int heads);
+}
+
+namespace {
+
+using namespace mla;
+
+// One error word per device: a file-scope device variable, so it exists as soon
+// as the library is loaded on a device and needs no allocation.
+__device__ int g_device_error;
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceState {
+  bool init = false;
+  int sm_count = 0;
+  int* err = nullptr;           // device address of g_device_error
+  void* ws = nullptr;           // workspace base
+  size_t ws_bytes = 0;
+  bool ws_external = false;     // set by mla_set_workspace
+  // timing
+  std::vector<cudaEvent_t> events;  // 4 per recorded call
+  int timed_calls = 0;
+};
+
+std::mutex g_mu;
+DeviceState g_dev[kMaxDevices];
+std::atomic<int> g_knobs[8];
+std::atomic<int> g_timing{0};
+thread_local char g_msg[512] = "";
+
+mla_status_t fail(mla_status_t s, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_msg, sizeof g_msg, fmt, ap);
+  va_end(ap);
+  return s;
+}
+
+mla_status_t cuda_fail(cudaError_t e, const char* what) {
+  return fail(MLA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+// Current device's state, initialised on first use (must hold g_mu).
+mla_status_t device_state(DeviceState** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) return fail(MLA_ERR_UNSUPPORTED, "device ordinal %d", dev);
+  DeviceState& d = g_dev[dev];
+  if (!d.init) {
+    e = cudaDeviceGetAttribute(&d.sm_count, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute");
+    e = cudaGetSymbolAddress(reinterpret_cast<void**>(&d.err), g_device_error);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(error word)");
+    d.init = true;
+  }
+  *out = &d;
+  return MLA_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Decode kernel choice: knob, else the tcgen05 kernel when it handles the shape.
+int pick_kernel(int heads) {
+  const int k = g_knobs[MLA_KNOB_DECODE_KERNEL].load();
+  if (k == 1) return 1;
+  if (k == 2) return decode_tc_supported(heads) ? 2 : -1;
+  return decode_tc_supported(heads) ? 2 : 1;
+}
+
+int num_workers_for(const DeviceState& d, int kernel, int heads) {
+  const int forced = g_knobs[MLA_KNOB_NUM_WORKERS].load();
+  if (forced > 0) return forced;
+  if (kernel == 2) return d.sm_count / 2;  // one CTA pair per worker
+  const int groups = (heads + decode_mma_heads_per_cta() - 1) / decode_mma_heads_per_cta();
+  return std::max(1, d.sm_count / groups);
+}
+
+mla_status_t ensure_workspace(DeviceState& d, size_t need, cudaStream_t stream) {
+  if (need <= d.ws_bytes) return MLA_OK;
+  if (d.ws_external)
+    return fail(MLA_ERR_WORKSPACE, "workspace of %zu bytes is smaller than the %zu bytes needed", d.ws_bytes, need);
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  cudaError_t e = cudaStreamIsCapturing(stream, &cs);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaStreamIsCapturing");
+  if (cs != cudaStreamCaptureStatusNone)
+    return fail(MLA_ERR_WORKSPACE, "workspace must grow to %zu bytes but the stream is capturing", need);
+  if (d.ws) {
+    e = cudaFree(d.ws);  // waits for work that may still use it
+    d.ws = nullptr;
+    d.ws_bytes = 0;
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFree(workspace)");
+  }
+  e = cudaMalloc(&d.ws, need);
+  if (e != cudaSuccess) {
+    d.ws = nullptr;
+    return cuda_fail(e, "cudaMalloc(workspace)");
+  }
+  d.ws_bytes = need;
+  return MLA_OK;
+}
+
+void record_event(DeviceState& d, int idx, cudaStream_t stream) {
+  if (!g_timing.load()) return;
+  const size_t i = (size_t)d.timed_calls * 4 + idx;
+  while (d.events.size() <= i) {
+    cudaEvent_t ev;
+    if (cudaEventCreate(&ev) != cudaSuccess) return;
+    d.events.push_back(ev);
+  }
+  cudaEventRecord(d.events[i], stream);
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* mla_status_string(mla_status_t s) {
+  switch (s) {
+    case MLA_OK: return "MLA_OK";
+    case MLA_ERR_INVALID_ARG: return "MLA_ERR_INVALID_ARG";
+    case MLA_ERR_UNSUPPORTED: return "MLA_ERR_UNSUPPORTED";
+    case MLA_ERR_WORKSPACE: return "MLA_ERR_WORKSPACE";
+    case MLA_ERR_CUDA: return "MLA_ERR_CUDA";
+    case MLA_ERR_DEVICE_BAD_PAGE: return "MLA_ERR_DEVICE_BAD_PAGE";
+    case MLA_ERR_DEVICE_TIMEOUT: return "MLA_ERR_DEVICE_TIMEOUT";
+  }
+  return "MLA_ERR_UNKNOWN";
+}
+
+const char* mla_last_error_message(void) { return g_msg; }
+
+mla_status_t mla_set_knob(mla_knob_t knob, int value) {
+  if ((int)knob < 0 || (int)knob >= 8) return fail(MLA_ERR_INVALID_ARG, "unknown knob %d", (int)knob);
+  if (value < 0) return fail(MLA_ERR_INVALID_ARG, "knob value %d < 0", value);
+  g_knobs[knob].store(value);
+  return MLA_OK;
+}
+
+int mla_get_knob(mla_knob_t knob) {
+  if ((int)knob < 0 || (int)knob >= 8) return -1;
+  return g_knobs[knob].load();
+}
+
+size_t mla_workspace_size(int batch, int heads, int max_blocks) {
+  (void)max_blocks;
+  if (batch <= 0 || heads <= 0) return 0;
+  std::lock_guard<std::mutex> lk(g_mu);
+  DeviceState* d = nullptr;
+  if (device_state(&d) != MLA_OK) return 0;
+  const int kernel = pick_kernel(heads);
+  const int P = num_workers_for(*d, kernel < 0 ? 1 : kernel, heads);
+  return carve_schedule(nullptr, batch, heads, P, nullptr);
+}
+
+mla_status_t mla_set_workspace(void* dev_ptr, size_t bytes) {
+  if (dev_ptr && (reinterpret_cast<uintptr_t>(dev_ptr) & 255u))
+    return fail(MLA_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+  std::lock_guard<std::mutex> lk(g_mu);
+  DeviceState* d = nullptr;
+  mla_status_t s = device_state(&d);
+  if (s != MLA_OK) return s;
+  cudaError_t e = cudaDeviceSynchronize();
+  if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceSynchronize");
+  if (d->ws && !d->ws_external) {
+    e = cudaFree(d->ws);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFree(workspace)");
+  }
+  d->ws = dev_ptr;
+  d->ws_bytes = dev_ptr ? bytes : 0;
+  d->ws_external = dev_ptr != nullptr;
+  return MLA_OK;
+}
+
+mla_status_t mla_get_device_error(mla_stream_t stream) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  DeviceState* d = nullptr;
+  mla_status_t s = device_state(&d);
+  if (s != MLA_OK) return s;
+  cudaError_t e = cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+  int v = 0;
+  e = cudaMemcpy(&v, d->err, sizeof(int), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(e, "read error word");
+  const int zero = 0;
+  e = cudaMemcpy(d->err, &zero, sizeof(int), cudaMemcpyHostToDevice);
+  if (e != cudaSuccess) return cuda_fail(e, "clear error word");
+  if (v == 0) return MLA_OK;
+  return v == MLA_ERR_DEVICE_TIMEOUT ? MLA_ERR_DEVICE_TIMEOUT : MLA_ERR_DEVICE_BAD_PAGE;
+}
+
+mla_status_t mla_decode(const void* q, const void* kv_cache, const int32_t* block_table,
+                        const int32_t* cache_seqlens, float* out, float* lse, int batch, int heads,
+                        int num_pages, int max_blocks, float softmax_scale, mla_stream_t stream_) {
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  if (batch < 0 || heads < 0 || max_blocks < 0 || num_pages < 0)
+    return fail(MLA_ERR_INVALID_ARG, "negative size (batch %d, heads %d, max_blocks %d, num_pages %d)", batch, heads,
+                max_blocks, num_pages);
+  if (batch == 0) return MLA_OK;
+  if (!q || !kv_cache || !cache_seqlens || !out || !lse)
+    return fail(MLA_ERR_INVALID_ARG, "null pointer argument");
+  if (heads < 1 || heads > MLA_MAX_HEADS) return fail(MLA_ERR_UNSUPPORTED, "heads = %d outside [1, 128]", heads);
+  if (max_blocks < 1) return fail(MLA_ERR_INVALID_ARG, "max_blocks must be >= 1");
+  if (block_table && num_pages < 1) return fail(MLA_ERR_INVALID_ARG, "paged cache with num_pages < 1");
+  if ((long long)batch * max_blocks > (1LL << 31) - 1 || (long long)max_blocks * MLA_PAGE_TOKENS > (1LL << 30))
+    return fail(MLA_ERR_UNSUPPORTED, "cache too large for 32-bit page indexing");
+  if (!aligned16(q) || !aligned16(kv_cache) || !aligned16(out))
+    return fail(MLA_ERR_INVALID_ARG, "q, kv_cache and out must be 16-byte aligned");
+  if ((reinterpret_cast<uintptr_t>(block_table) & 3u) || (reinterpret_cast<uintptr_t>(cache_seqlens) & 3u) ||
+      (reinterpret_cast<uintptr_t>(lse) & 3u))
+    return fail(MLA_ERR_INVALID_ARG, "int32/fp32 arrays must be 4-byte aligned");
+  if (!std::isfinite(softmax_scale)) return fail(MLA_ERR_INVALID_ARG, "softmax_scale is not finite");
+
+  std::lock_guard<std::mutex> lk(g_mu);
+  DeviceState* d = nullptr;
+  mla_status_t s = device_state(&d);
+  if (s != MLA_OK) return s;
+  const int kernel = pick_kernel(heads);
+  if (kernel < 0) return fail(MLA_ERR_UNSUPPORTED, "requested decode kernel does not handle heads = %d", heads);
+  const int P = num_workers_for(*d, kernel, heads);
+  const size_t need = carve_schedule(nullptr, batch, heads, P, nullptr);
+  s = ensure_workspace(*d, need, stream);
+  if (s != MLA_OK) return s;
+
+  DecodeArgs a{};
+  a.q = static_cast<const __nv_bfloat16*>(q);
+  a.kv = static_cast<const __nv_bfloat16*>(kv_cache);
+  a.block_table = block_table;
+  a.seqlens = cache_seqlens;
+  a.out = out;
+  a.lse = lse;
+  a.batch = batch;
+  a.heads = heads;
+  a.num_pages = num_pages;
+  a.max_blocks = max_blocks;
+  a.scale = softmax_scale;
+  a.err = d->err;
+  carve_schedule(d->ws, batch, heads, P, &a.sched);
+  a.wait_limit = g_knobs[MLA_KNOB_WAIT_LIMIT].load() > 0 ? g_knobs[MLA_KNOB_WAIT_LIMIT].load() : (1 << 26);
+  a.withhold_arrive = g_knobs[MLA_KNOB_WITHHOLD_ARRIVE].load();
+  const int min_pages = g_knobs[MLA_KNOB_MIN_PAGES].load() > 0 ? g_knobs[MLA_KNOB_MIN_PAGES].load() : 4;
+
+  record_event(*d, 0, stream);
+  cudaError_t e = launch_schedule(cache_seqlens, batch, max_blocks, min_pages, a.sched, d->err, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "schedule launch");
+  record_event(*d, 1, stream);
+  e = kernel == 2 ? launch_decode_tc(a, stream) : launch_decode_mma(a, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "decode launch");
+  record_event(*d, 2, stream);
+  e = launch_combine(a, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "combine launch");
+  record_event(*d, 3, stream);
+  if (g_timing.load()) d->timed_calls++;
+  return MLA_OK;
+}
+
+mla_status_t mla_absorb_q(const void* q_nope, const void* q_rope, const void* w_uk, void* q_out, int batch,
+                          int heads, mla_stream_t stream) {
+  if (batch < 0 || heads < 0) return fail(MLA_ERR_INVALID_ARG, "negative size");
+  if (batch == 0) return MLA_OK;
+  if (!q_nope || !q_rope || !w_uk || !q_out) return fail(MLA_ERR_INVALID_ARG, "null pointer argument");
+  if (heads < 1 || heads > MLA_MAX_HEADS) return fail(MLA_ERR_UNSUPPORTED, "heads = %d outside [1, 128]", heads);
+  if (!aligned16(q_nope) || !aligned16(q_rope) || !aligned16(w_uk) || !aligned16(q_out))
+    return fail(MLA_ERR_INVALID_ARG, "absorb_q operands must be 16-byte aligned");
+  cudaError_t e = launch_absorb_q(static_cast<const __nv_bfloat16*>(q_nope), static_cast<const __nv_bfloat16*>(q_rope),
+                                  static_cast<const __nv_bfloat16*>(w_uk), static_cast<__nv_bfloat16*>(q_out), batch,
+                                  heads, reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? MLA_OK : cuda_fail(e, "absorb_q launch");
+}
+
+mla_status_t mla_absorb_o(const float* out_latent, const void* w_uv, float* out, int batch, int heads,
+                          mla_stream_t stream) {
+  if (batch < 0 || heads < 0) return fail(MLA_ERR_INVALID_ARG, "negative size");
+  if (batch == 0) return MLA_OK;
+  if (!out_latent || !w_uv || !out) return fail(MLA_ERR_INVALID_ARG, "null pointer argument");
+  if (heads < 1 || heads > MLA_MAX_HEADS) return fail(MLA_ERR_UNSUPPORTED, "heads = %d outside [1, 128]", heads);
+  if (!aligned16(out_latent) || !aligned16(w_uv) || !aligned16(out))
+    return fail(MLA_ERR_INVALID_ARG, "absorb_o operands must be 16-byte aligned");
+  cudaError_t e = launch_absorb_o(out_latent, static_cast<const __nv_bfloat16*>(w_uv), out, batch, heads,
+                                  reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? MLA_OK : cuda_fail(e, "absorb_o launch");
+}
+
+mla_status_t mla_timing_enable(int enable) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  DeviceState* d = nullptr;
+  mla_status_t s = device_state(&d);
+  if (s != MLA_OK) return s;
+  d->timed_calls = 0;
+  g_timing.store(enable ? 1 : 0);
+  return MLA_OK;
+}
+
+mla_status_t mla_timing_read(float ms[3], int* calls) {
+  if (!ms || !calls) return fail(MLA_ERR_INVALID_ARG, "null pointer argument");
+  std::lock_guard<std::mutex> lk(g_mu);
+  DeviceState* d = nullptr;
+  mla_status_t s = device_state(&d);
+  if (s != MLA_OK) return s;
+  ms[0] = ms[1] = ms[2] = 0.f;
+  *calls = d->timed_calls;
+  if (d->timed_calls > 0) {
+    cudaError_t e = cudaEventSynchronize(d->events[(size_t)d->timed_calls * 4 - 1]);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaEventSynchronize");
+    for (int c = 0; c < d->timed_calls; ++c) {
+      for (int k = 0; k < 3; ++k) {
+        float t = 0.f;
+        e = cudaEventElapsedTime(&t, d->events[(size_t)c * 4 + k], d->events[(size_t)c * 4 + k + 1]);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaEventElapsedTime");
+        ms[k] += t;
+      }
+    }
+  }
+  d->timed_calls = 0;
+  return MLA_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,73 @@
+// Host-side interface between the C-ABI layer (api.cu) and the kernel files.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "mla.h"
+
+namespace mla {
+
+// Split schedule, written on the device by the schedule kernel.
+//
+// The pages of all sequences are laid end to end (sequence-major); worker w takes
+// the contiguous range [w*q, min((w+1)*q, N)) of that list, q = max(ceil(N/P),
+// min_pages).  A worker's range covers a tail of its first sequence, whole middle
+// sequences and a head of its last one.  A sequence that one worker covers
+// entirely is written straight to out/lse; otherwise every worker writes its piece
+// (normalised partial output and its lse) to a partial slot -- slot w when the
+// sequence is the worker's first, slot P + w otherwise -- and the combine kernel
+// merges the pieces by their lse.  Everything depends only on the sequence lengths,
+// the batch size and P.
+struct WorkerRange {
+  int b0, p0;  // first sequence and its first page
+  int b1, p1;  // last sequence and one past its last page (b0 < 0: no work)
+};
+
+struct SeqInfo {
+  int first_worker;  // worker holding the sequence's first page
+  int num_pieces;    // workers covering it; 0 = empty sequence; -1 = invalid length
+};
+
+struct Schedule {
+  WorkerRange* ranges;  // [P]
+  int* seq_start;       // [B + 1] prefix sums of pages per sequence
+  SeqInfo* seq;         // [B]
+  int* quota;           // [1] pages per worker q
+  float* part_lse;      // [2P, H]  (natural-log lse of each piece)
+  float* part_o;        // [2P, H, 512] normalised partial outputs
+  int num_workers;      // P
+};
+
+// Workspace carve-up; `base` may be null to just compute the size.
+size_t carve_schedule(void* base, int batch, int heads, int num_workers, Schedule* s);
+
+struct DecodeArgs {
+  const __nv_bfloat16* q;
+  const __nv_bfloat16* kv;
+  const int32_t* block_table;  // null = contiguous cache
+  const int32_t* seqlens;
+  float* out;
+  float* lse;
+  int batch, heads, num_pages, max_blocks;
+  float scale;
+  int* err;
+  Schedule sched;
+  int wait_limit;       // bounded-wait spin limit (tcgen05 kernel)
+  int withhold_arrive;  // test hook (tcgen05 kernel)
+};
+
+cudaError_t launch_schedule(const int32_t* seqlens, int batch, int max_blocks, int min_pages,
+                            const Schedule& s, int* err, cudaStream_t stream);
+cudaError_t launch_decode_mma(const DecodeArgs& a, cudaStream_t stream);
+int decode_mma_heads_per_cta();
+cudaError_t launch_combine(const DecodeArgs& a, cudaStream_t stream);
+cudaError_t launch_absorb_q(const __nv_bfloat16* q_nope, const __nv_bfloat16* q_rope,
+                            const __nv_bfloat16* w_uk, __nv_bfloat16* q_out, int batch, int heads,
+                            cudaStream_t stream);
+cudaError_t launch_absorb_o(const float* out_latent, const __nv_bfloat16* w_uv, float* out, int batch,
+                            int heads, cudaStream_t stream);
+
+}  // namespace mla

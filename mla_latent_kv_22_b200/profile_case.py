@@ -1,0 +1,43 @@
+"""Runs mla_decode on a synthetic paged case a few times: the command to put
+under a profiler (ncu) for a capture smaller than the benchmark workload.
+
+    python -m mla_latent_kv_22_b200.profile_case --batch 32 --seqlen 4096 --steps 3
+"""
+import argparse
+import math
+
+import numpy as np
+import torch
+
+import mla_latent_kv_22_b200 as M
+import mla_synth as S
+
+
+def main() -> None:
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--batch", type=int, default=32)
+    ap.add_argument("--heads", type=int, default=128)
+    ap.add_argument("--seqlen", type=int, default=4096)
+    ap.add_argument("--steps", type=int, default=3)
+    ap.add_argument("--kernel", type=int, default=0, help="0 auto, 1 mma.sync, 2 tcgen05")
+    a = ap.parse_args()
+    M.mla_set_knob("decode_kernel", a.kernel)
+    case = S.make_decode_case(a.batch, a.heads, a.seqlen, seed=3, poison=False, latent_std=0.5)
+    dev = lambda x: torch.from_numpy(np.ascontiguousarray(x).view(np.int16)).view(torch.bfloat16).cuda()
+    q, kv = dev(case.q), dev(case.kv_cache)
+    bt = torch.from_numpy(case.block_table).cuda()
+    sl = torch.from_numpy(case.cache_seqlens).cuda()
+    out = torch.empty(a.batch, a.heads, 512, device="cuda")
+    lse = torch.empty(a.batch, a.heads, device="cuda")
+    for _ in range(a.steps):
+        M.mla_decode(q, kv, bt, sl, out, lse, 1.0 / math.sqrt(192.0))
+    torch.cuda.synchronize()
+    status = M.mla_get_device_error()
+    print(f"profile_case: B={a.batch} H={a.heads} T={a.seqlen} steps={a.steps} device_error={status} "
+          f"finite={bool(torch.isfinite(out).all())}")
+    if status:
+        raise SystemExit(1)
+
+
+if __name__ == "__main__":
+    main()
