@@ -62,21 +62,23 @@ def measured_peaks() -> tuple[dict, str]:
     return {"hbm_gbs": FALLBACK_HBM_GBS, "bf16_tflops": FALLBACK_BF16_TFLOPS}, "fallback"
 
 
-def decode_source_hash() -> str:
-    """Hash of the decode kernels' sources, to tie an ncu traffic figure to them."""
+def decode_source_hash(kernel: str) -> str:
+    """Hash of the sources of the decode kernel that ran (and the headers it uses),
+    to tie an ncu traffic figure to exactly that code."""
+    files = {"tcgen05": ["decode_tc.cu", "sm100_ptx.cuh"], "mma.sync": ["decode_mma.cu"]}[kernel]
+    files += ["mla_device.cuh", "mla_internal.h"]
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "mla_latent_kv_22_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
-        if name.startswith("decode") or name in ("mla_device.cuh", "combine.cu", "schedule.cu"):
-            with open(os.path.join(csrc, name), "rb") as f:
-                h.update(name.encode() + f.read())
+    for name in files:
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode() + f.read())
     return h.hexdigest()[:16]
 
 
-def ncu_traffic(kernel_hash: str):
-    """DRAM bytes per decode launch from the committed ncu summary, if it was taken
-    on the current sources (else None)."""
-    p = os.path.join(ROOT, "profiles", "decode_headline_traffic.json")
+def ncu_traffic(kernel: str, kernel_hash: str):
+    """DRAM bytes per decode launch (headline workload) from the committed ncu summary,
+    if it was taken on the current sources of that kernel (else None)."""
+    p = os.path.join(ROOT, "profiles", f"decode_{kernel.replace('.', '')}_headline_traffic.json")
     if not os.path.exists(p):
         return None
     with open(p) as f:
@@ -131,10 +133,18 @@ _REASONS = {
 
 
 class ClockSampler:
+    """Polls SM clock and clock-event reasons through NVML from a host thread.
+
+    Every sample carries a host timestamp, so the summary can keep only the samples
+    taken inside the device-timed region; when that region is too short for three
+    samples, it reports all samples of the GPU-busy window (warm-up, timed and
+    end-to-end loops, all under the same load) and says so."""
+
     def __init__(self, device_index: int):
-        self.samples: list[tuple[int, int, int]] = []
+        self.samples: list[tuple[float, int, int]] = []
         self._stop = threading.Event()
         self._ok = False
+        self.window = None
         try:
             import pynvml
             pynvml.nvmlInit()
@@ -152,35 +162,41 @@ class ClockSampler:
             try:
                 sm = nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM)
                 rs = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
-                util = nv.nvmlDeviceGetUtilizationRates(self._h).gpu
-                self.samples.append((sm, rs, util))
+                self.samples.append((time.perf_counter(), sm, rs))
             except Exception:
-                pass
-            time.sleep(0.002)
+                time.sleep(0.001)
 
-    def __enter__(self):
+    def start(self):
         if self._ok:
             self._t = threading.Thread(target=self._run, daemon=True)
             self._t.start()
         return self
 
-    def __exit__(self, *exc):
+    def stop(self):
         if self._ok:
             self._stop.set()
             self._t.join()
 
+    def mark(self, t0: float, t1: float):
+        self.window = (t0, t1)
+
     def summary(self) -> dict:
         if not self._ok:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0, "error": getattr(self, "error", "")}
-        if not self.samples:
+        picked, where = self.samples, "warm-up + timed + end-to-end loops"
+        if self.window is not None:
+            inside = [x for x in self.samples if self.window[0] <= x[0] <= self.window[1]]
+            if len(inside) >= 3:
+                picked, where = inside, "timed region"
+        if not picked:
             return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0}
-        mhz = [s[0] for s in self.samples]
+        mhz = [x[1] for x in picked]
         mask = 0
-        for s in self.samples:
-            mask |= s[1]
+        for x in picked:
+            mask |= x[2]
         reasons = [n for bit, n in _REASONS.items() if mask & bit and n != "gpu_idle"]
         return {"sm_mhz": statistics.median(mhz), "sm_max_mhz": self.max_mhz, "reasons": reasons,
-                "samples": len(self.samples), "sm_mhz_min": min(mhz)}
+                "samples": len(picked), "sm_mhz_min": min(mhz), "window": where}
 
 
 # ---------------------------------------------------------------------------
@@ -270,6 +286,7 @@ def run_ours(args) -> None:
     def step():
         M.mla_decode(q, kv, bt, sl, out, lse, case.softmax_scale, stream=stream)
 
+    clk = ClockSampler(local_rank).start()
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize(device)
@@ -281,12 +298,13 @@ def run_ours(args) -> None:
     M.mla_timing_enable(True)
     barrier(dist, device)
     torch.cuda.synchronize(device)
-    with ClockSampler(local_rank) as clk:
-        e0.record(stream)
-        for _ in range(args.steps):
-            step()
-        e1.record(stream)
-        torch.cuda.synchronize(device)
+    h0 = time.perf_counter()
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize(device)
+    clk.mark(h0, time.perf_counter())
     barrier(dist, device)
     ms_total = e0.elapsed_time(e1)
     kern_ms, calls = M.mla_timing_read()
@@ -322,6 +340,7 @@ def run_ours(args) -> None:
     f1.record(stream)
     torch.cuda.synchronize(device)
     barrier(dist, device)
+    clk.stop()
     e2e_ms = max_over_ranks(f0.elapsed_time(f1) / args.steps, dist, device)
     h2d = q_h.numel() * 2 + bt_h.numel() * 4 + sl_h.numel() * 4
     d2h = out_h.numel() * 4 + lse_h.numel() * 4
@@ -338,8 +357,9 @@ def run_ours(args) -> None:
     achieved = alg_bytes / (dec_ms * 1e-3) / 1e9  # GB/s
     hbm_peak = float(peaks["hbm_gbs"])
     roofline_us = max(alg_bytes / (hbm_peak * 1e9), flops / (float(peaks["bf16_tflops"]) * 1e12)) * 1e6
-    khash = decode_source_hash()
-    traffic = ncu_traffic(khash)
+    kernel = {1: "mma.sync", 2: "tcgen05"}[M.mla_selected_decode_kernel(H)]
+    khash = decode_source_hash(kernel)
+    traffic = ncu_traffic(kernel, khash)
     us_step = ms_step * 1e3
     line = {
         "metric": METRIC, "value": us_step, "unit": UNIT, "n_gpus": world, "steps": args.steps,
@@ -356,12 +376,12 @@ def run_ours(args) -> None:
                       "combine": kern_ms[2] / max(calls, 1) * 1e3},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
                      "frac": achieved / hbm_peak, "traffic": traffic,
-                     "peak_kind": peak_kind, "kernel": "decode (split-KV)",
+                     "peak_kind": peak_kind, "kernel": f"decode ({kernel})",
                      "algorithmic_bytes_per_launch": alg_bytes, "source_hash": khash},
         "gpu_launches": 3 * args.steps,
         "e2e": {"value": e2e_ms * 1e3, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "clocks": clk.summary(),
-        "decode_kernel": {0: "auto", 1: "mma.sync", 2: "tcgen05"}[M.mla_get_knob("decode_kernel")],
+        "decode_kernel": kernel,
     }
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline()

@@ -165,12 +165,15 @@ typedef enum {
   MLA_KNOB_NUM_WORKERS = 0,     /* > 0: force the number of split workers; 0 = auto         */
   MLA_KNOB_MIN_PAGES = 1,       /* > 0: minimum pages per worker; 0 = auto                  */
   MLA_KNOB_DECODE_KERNEL = 2,   /* 0 = auto, 1 = mma.sync kernel, 2 = tcgen05 kernel        */
-  MLA_KNOB_WAIT_LIMIT = 3,      /* > 0: spin limit of bounded waits (tests shorten it)      */
+  MLA_KNOB_WAIT_LIMIT = 3,      /* > 0: time limit of bounded device waits in ms; 0 = 2000  */
   MLA_KNOB_WITHHOLD_ARRIVE = 4  /* 1: the tcgen05 kernel's producer skips one arrive, so the
                                    consumer's bounded wait must run out (timeout test)      */
 } mla_knob_t;
 mla_status_t mla_set_knob(mla_knob_t knob, int value);
 int mla_get_knob(mla_knob_t knob);
+/* Which decode kernel mla_decode runs for `heads` under the current knobs:
+   1 = mma.sync kernel, 2 = tcgen05 kernel, -1 = none handles it. */
+int mla_selected_decode_kernel(int heads);
 
 /*
  * Per-launch device timing.  While enabled, every mla_decode records CUDA events

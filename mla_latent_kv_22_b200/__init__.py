@@ -4,7 +4,7 @@ Argument marshalling only.  Every function takes torch tensors, checks dtype,
 shape, device and contiguity, and passes raw pointers, sizes and the current CUDA
 stream to the C ABI of the same name (include/mla.h); every step of the
 computation runs in the library's CUDA kernels.  Importing fails loudly when the
-library has not been built (``python -m mla_latent_kv_22_b200.build``); there is
+library has not been built (``python mla_latent_kv_22_b200/build.py``); there is
 no fallback.
 """
 from __future__ import annotations
@@ -16,7 +16,8 @@ import torch
 
 __all__ = [
     "MlaError", "mla_decode", "mla_absorb_q", "mla_absorb_o", "mla_workspace_size", "mla_set_workspace",
-    "mla_get_device_error", "mla_status_string", "mla_set_knob", "mla_get_knob", "mla_timing_enable",
+    "mla_get_device_error", "mla_status_string", "mla_set_knob", "mla_get_knob", "mla_selected_decode_kernel",
+    "mla_timing_enable",
     "mla_timing_read", "lib", "LIB_PATH", "KNOB", "STATUS",
 ]
 
@@ -40,7 +41,7 @@ class MlaError(RuntimeError):
 
 def _load() -> ctypes.CDLL:
     if not os.path.exists(LIB_PATH):
-        raise ImportError(f"{LIB_PATH} is missing: build it with `python -m mla_latent_kv_22_b200.build` "
+        raise ImportError(f"{LIB_PATH} is missing: build it with `python mla_latent_kv_22_b200/build.py` "
                           "(nvcc, sm_100a); there is no fallback implementation")
     L = ctypes.CDLL(LIB_PATH)
     vp, i32, f32, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
@@ -55,6 +56,7 @@ def _load() -> ctypes.CDLL:
         "mla_last_error_message": ([], ctypes.c_char_p),
         "mla_set_knob": ([i32, i32], i32),
         "mla_get_knob": ([i32], i32),
+        "mla_selected_decode_kernel": ([i32], i32),
         "mla_timing_enable": ([i32], i32),
         "mla_timing_read": ([ctypes.POINTER(ctypes.c_float), ctypes.POINTER(ctypes.c_int)], i32),
     }
@@ -169,6 +171,11 @@ def mla_set_knob(name: str, value: int) -> None:
 
 def mla_get_knob(name: str) -> int:
     return int(lib.mla_get_knob(KNOB[name]))
+
+
+def mla_selected_decode_kernel(heads: int) -> int:
+    """1 = mma.sync kernel, 2 = tcgen05 kernel (what mla_decode runs for ``heads`` now)."""
+    return int(lib.mla_selected_decode_kernel(int(heads)))
 
 
 def mla_timing_enable(enable: bool = True) -> None:

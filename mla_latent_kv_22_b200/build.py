@@ -1,6 +1,8 @@
 """Builds libmla.so in-tree with nvcc for sm_100a (B200).
 
-    python -m mla_latent_kv_22_b200.build [--force] [--verbose]
+    python mla_latent_kv_22_b200/build.py [--force] [--verbose] [--ptxas]
+
+(Run it as a file, not with ``-m``: importing the package loads the library.)
 """
 from __future__ import annotations
 

@@ -18,6 +18,7 @@ namespace mla {
 // Defined in decode_tc.cu.
 cudaError_t launch_decode_tc(const DecodeArgs& a, cudaStream_t stream);
 bool decode_tc_supported(int heads);
+int decode_tc_max_workers(int sm_count);
 }
 
 namespace {
@@ -85,13 +86,13 @@ int pick_kernel(int heads) {
   const int k = g_knobs[MLA_KNOB_DECODE_KERNEL].load();
   if (k == 1) return 1;
   if (k == 2) return decode_tc_supported(heads) ? 2 : -1;
-  return decode_tc_supported(heads) ? 2 : 1;
+  return 1;
 }
 
 int num_workers_for(const DeviceState& d, int kernel, int heads) {
   const int forced = g_knobs[MLA_KNOB_NUM_WORKERS].load();
   if (forced > 0) return forced;
-  if (kernel == 2) return d.sm_count / 2;  // one CTA pair per worker
+  if (kernel == 2) return std::max(1, std::min(d.sm_count / 2, decode_tc_max_workers(d.sm_count)));  // CTA pairs
   const int groups = (heads + decode_mma_heads_per_cta() - 1) / decode_mma_heads_per_cta();
   return std::max(1, d.sm_count / groups);
 }
@@ -160,6 +161,11 @@ mla_status_t mla_set_knob(mla_knob_t knob, int value) {
 int mla_get_knob(mla_knob_t knob) {
   if ((int)knob < 0 || (int)knob >= 8) return -1;
   return g_knobs[knob].load();
+}
+
+int mla_selected_decode_kernel(int heads) {
+  if (heads < 1 || heads > MLA_MAX_HEADS) return -1;
+  return pick_kernel(heads);
 }
 
 size_t mla_workspace_size(int batch, int heads, int max_blocks) {
@@ -256,7 +262,7 @@ mla_status_t mla_decode(const void* q, const void* kv_cache, const int32_t* bloc
   a.scale = softmax_scale;
   a.err = d->err;
   carve_schedule(d->ws, batch, heads, P, &a.sched);
-  a.wait_limit = g_knobs[MLA_KNOB_WAIT_LIMIT].load() > 0 ? g_knobs[MLA_KNOB_WAIT_LIMIT].load() : (1 << 26);
+  a.wait_limit = g_knobs[MLA_KNOB_WAIT_LIMIT].load() > 0 ? g_knobs[MLA_KNOB_WAIT_LIMIT].load() : 2000;  // ms
   a.withhold_arrive = g_knobs[MLA_KNOB_WITHHOLD_ARRIVE].load();
   const int min_pages = g_knobs[MLA_KNOB_MIN_PAGES].load() > 0 ? g_knobs[MLA_KNOB_MIN_PAGES].load() : 4;
 

@@ -55,7 +55,7 @@ struct DecodeArgs {
   float scale;
   int* err;
   Schedule sched;
-  int wait_limit;       // bounded-wait spin limit (tcgen05 kernel)
+  int wait_limit;       // bounded-wait time limit in milliseconds (tcgen05 kernel)
   int withhold_arrive;  // test hook (tcgen05 kernel)
 };
 
