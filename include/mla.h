@@ -132,6 +132,29 @@ mla_status_t mla_absorb_q(const void* q_nope, const void* q_rope, const void* w_
 mla_status_t mla_absorb_o(const float* out_latent, const void* w_uv, float* out,
                           int batch, int heads, mla_stream_t stream);
 
+/*
+ * mla_decode_noalloc -- mla_decode for callers that cannot allocate device memory.
+ *
+ * The pages have no counterpart of this call; it exists for callers such as a
+ * serving runtime that has already reserved all device memory for its own pool,
+ * code running while a stream is captured into a CUDA graph (where cudaMalloc is
+ * not allowed), or latency-critical paths that cannot absorb cudaMalloc's implicit
+ * device synchronisation.  Arguments, layouts, results and errors are those of
+ * mla_decode.  Instead of the workspace, it uses one 32 MiB static device array
+ * that each GPU loading the library holds until exit; it never calls cudaMalloc or
+ * cudaFree.  Sizes whose split partials and schedule do not fit are rejected with
+ * MLA_ERR_UNSUPPORTED before any launch; to fit, it may split over fewer workers
+ * than mla_decode, so results match mla_decode within rounding, not bit for bit.
+ * The first call on a device looks up the array's device address; make it before
+ * any stream capture.  All calls on a device share the array (it keeps the last
+ * call's contents; nothing in it must start at zero): calls that overlap on the GPU
+ * race and must be serialised by the caller.
+ */
+mla_status_t mla_decode_noalloc(const void* q, const void* kv_cache, const int32_t* block_table,
+                                const int32_t* cache_seqlens, float* out, float* lse,
+                                int batch, int heads, int num_pages, int max_blocks,
+                                float softmax_scale, mla_stream_t stream);
+
 /* Bytes of workspace mla_decode needs on the current device for these sizes. */
 size_t mla_workspace_size(int batch, int heads, int max_blocks);
 

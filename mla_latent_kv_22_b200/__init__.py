@@ -15,7 +15,7 @@ import os
 import torch
 
 __all__ = [
-    "MlaError", "mla_decode", "mla_absorb_q", "mla_absorb_o", "mla_workspace_size", "mla_set_workspace",
+    "MlaError", "mla_decode", "mla_decode_noalloc", "mla_absorb_q", "mla_absorb_o", "mla_workspace_size", "mla_set_workspace",
     "mla_get_device_error", "mla_status_string", "mla_set_knob", "mla_get_knob", "mla_selected_decode_kernel",
     "mla_timing_enable",
     "mla_timing_read", "lib", "LIB_PATH", "KNOB", "STATUS",
@@ -47,6 +47,7 @@ def _load() -> ctypes.CDLL:
     vp, i32, f32, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
     sig = {
         "mla_decode": ([vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, f32, vp], i32),
+        "mla_decode_noalloc": ([vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, f32, vp], i32),
         "mla_absorb_q": ([vp, vp, vp, vp, i32, i32, vp], i32),
         "mla_absorb_o": ([vp, vp, vp, i32, i32, vp], i32),
         "mla_workspace_size": ([i32, i32, i32], sz),
@@ -121,6 +122,39 @@ def mla_decode(q, kv_cache, block_table, cache_seqlens, out, lse, softmax_scale:
         max_blocks, num_pages, bt = int(block_table.shape[1]), int(kv_cache.shape[0]), block_table.data_ptr()
     _check(lib.mla_decode(q.data_ptr(), kv_cache.data_ptr(), bt, cache_seqlens.data_ptr(), out.data_ptr(),
                           lse.data_ptr(), B, H, num_pages, max_blocks, float(softmax_scale), _stream(stream)))
+
+
+def _noalloc_args(q, kv_cache, block_table, cache_seqlens, out, lse):
+    if q.dim() == 4 and q.shape[1] == 1:  # [B, 1, H, 576] (s_q = 1)
+        q = q.view(q.shape[0], q.shape[2], q.shape[3])
+    B, H = int(q.shape[0]), int(q.shape[1])
+    _need(q, "q", torch.bfloat16, (B, H, D_QK))
+    _need(cache_seqlens, "cache_seqlens", torch.int32, (B,))
+    _need(out, "out", torch.float32, (B, H, D_LATENT))
+    _need(lse, "lse", torch.float32, (B, H))
+    if block_table is None:
+        _need(kv_cache, "kv_cache", torch.bfloat16)
+        if kv_cache.dim() != 3 or kv_cache.shape[0] != B or kv_cache.shape[2] != D_QK or kv_cache.shape[1] % PAGE:
+            raise ValueError("contiguous kv_cache must be [B, Tcap, 576] with Tcap % 64 == 0")
+        max_blocks, num_pages, bt = int(kv_cache.shape[1]) // PAGE, 0, None
+    else:
+        _need(block_table, "block_table", torch.int32)
+        _need(kv_cache, "kv_cache", torch.bfloat16)
+        if kv_cache.dim() != 3 or tuple(kv_cache.shape[1:]) != (PAGE, D_QK):
+            raise ValueError("paged kv_cache must be [num_pages, 64, 576]")
+        if block_table.dim() != 2 or block_table.shape[0] != B:
+            raise ValueError("block_table must be [B, max_blocks]")
+        max_blocks, num_pages, bt = int(block_table.shape[1]), int(kv_cache.shape[0]), block_table.data_ptr()
+    return (q.data_ptr(), kv_cache.data_ptr(), bt, cache_seqlens.data_ptr(), out.data_ptr(), lse.data_ptr(), B, H,
+            num_pages, max_blocks)
+
+
+def mla_decode_noalloc(q, kv_cache, block_table, cache_seqlens, out, lse, softmax_scale: float,
+                       stream=None) -> None:
+    """mla_decode for callers that cannot allocate device memory: same arguments and
+    results, scratch from the library's static 32 MiB device array (see include/mla.h)."""
+    args = _noalloc_args(q, kv_cache, block_table, cache_seqlens, out, lse)
+    _check(lib.mla_decode_noalloc(*args, float(softmax_scale), _stream(stream)))
 
 
 def mla_absorb_q(q_nope, q_rope, w_uk, q_out, stream=None) -> None:

@@ -134,6 +134,26 @@ void record_event(DeviceState& d, int idx, cudaStream_t stream) {
 
 }  // namespace
 
+namespace mla {
+// The per-device facts mla_decode uses (decode kernel, worker count, error word),
+// for the allocation-free entry point in noalloc.cu.
+mla_status_t decode_plan(int heads, int* kernel, int* num_workers, int** err_word) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  DeviceState* d = nullptr;
+  mla_status_t s = device_state(&d);
+  if (s != MLA_OK) return s;
+  *kernel = pick_kernel(heads);
+  if (*kernel < 0) return fail(MLA_ERR_UNSUPPORTED, "requested decode kernel does not handle heads = %d", heads);
+  *num_workers = num_workers_for(*d, *kernel, heads);
+  *err_word = d->err;
+  return MLA_OK;
+}
+
+mla_status_t record_error(mla_status_t s, const char* msg) { return fail(s, "%s", msg); }
+
+int knob_value(int knob) { return (knob >= 0 && knob < 8) ? g_knobs[knob].load() : 0; }
+}  // namespace mla
+
 extern "C" {
 
 const char* mla_status_string(mla_status_t s) {

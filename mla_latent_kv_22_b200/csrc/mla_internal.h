@@ -70,4 +70,11 @@ cudaError_t launch_absorb_q(const __nv_bfloat16* q_nope, const __nv_bfloat16* q_
 cudaError_t launch_absorb_o(const float* out_latent, const __nv_bfloat16* w_uv, float* out, int batch,
                             int heads, cudaStream_t stream);
 
+// Defined in api.cu: the per-device decode plan, the thread's last-error text,
+// and raw knob values.
+mla_status_t decode_plan(int heads, int* kernel, int* num_workers, int** err_word);
+mla_status_t record_error(mla_status_t s, const char* msg);
+int knob_value(int knob);
+cudaError_t launch_decode_tc(const DecodeArgs& a, cudaStream_t stream);
+
 }  // namespace mla
