@@ -269,6 +269,7 @@ def run_ours(args) -> None:
     import mla_synth as S
 
     rank, local_rank, world = dist_env()
+    M.mla_set_knob("decode_kernel", {"auto": 0, "mma.sync": 1, "tcgen05": 2}[args.kernel])
     torch.cuda.set_device(local_rank)
     device = torch.device("cuda", local_rank)
     dist = init_dist("nccl")
@@ -397,6 +398,8 @@ def main() -> None:
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--kernel", choices=["auto", "mma.sync", "tcgen05"], default="auto",
+                    help="decode kernel (default: the library's choice)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

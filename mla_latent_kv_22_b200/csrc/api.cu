@@ -86,7 +86,7 @@ int pick_kernel(int heads) {
   const int k = g_knobs[MLA_KNOB_DECODE_KERNEL].load();
   if (k == 1) return 1;
   if (k == 2) return decode_tc_supported(heads) ? 2 : -1;
-  return 1;
+  return decode_tc_supported(heads) ? 2 : 1;
 }
 
 int num_workers_for(const DeviceState& d, int kernel, int heads) {

@@ -24,9 +24,11 @@ def oracle_for(case, batch=None, heads=None):
                             batch=batch, heads=heads)
 
 
-@pytest.fixture(autouse=True)
-def _reset_knobs():
-    yield
+@pytest.fixture(autouse=True, params=[1, 2], ids=["mma", "tcgen05"])
+def kernel(request):
+    """Every test runs on both decode kernels."""
+    M.mla_set_knob("decode_kernel", request.param)
+    yield request.param
     for k in ("num_workers", "min_pages", "decode_kernel", "wait_limit", "withhold_arrive"):
         M.mla_set_knob(k, 0)
 
@@ -175,3 +177,21 @@ def test_kernel_timing_hook():
     ms, calls = M.mla_timing_read()
     M.mla_timing_enable(False)
     assert calls == 3 and all(x > 0 for x in ms)
+
+
+def test_bounded_wait_times_out_and_context_survives(kernel):
+    """A wait that nothing will satisfy (the producer withholds one page's arrival)
+    must end in MLA_ERR_DEVICE_TIMEOUT within the limit, without a trap or hang,
+    and the next call must run normally."""
+    if kernel != 2:
+        pytest.skip("only the tcgen05 kernel has mbarrier waits")
+    case = S.make_decode_case(4, 128, 1000, seed=46, poison=True)
+    dev = upload(case)
+    M.mla_set_knob("wait_limit", 50)
+    M.mla_set_knob("withhold_arrive", 1)
+    _, _, err = run_decode(case, dev)
+    assert err == 6  # MLA_ERR_DEVICE_TIMEOUT
+    M.mla_set_knob("withhold_arrive", 0)
+    out, lse, err = run_decode(case, dev)
+    assert err == 0
+    assert_close(out, lse, *oracle_for(case), "after a timeout")
