@@ -9,27 +9,35 @@
 // it: CTA r keeps O[:, 256r : 256r+256) and contracts the scores over its own dims
 // (latent [256r, 256r+256) plus rope [512+32r, 512+32r+32)).  Each CTA therefore
 // loads only its part of every row (HBM and L2 traffic 1x), computes a partial S,
-// and the two partials are exchanged through distributed shared memory and added in
-// the same order on both sides, so both CTAs run an identical softmax.
+// and the two fp32 partials are exchanged through distributed shared memory by bulk
+// copies (32 KB per page each way) and added in the same order on both sides, so
+// both CTAs run a bit-identical softmax.
+//
+// Pipeline.  The exchange has a long latency, so the softmax threads are software
+// pipelined: in each iteration they first send page j+1's partial (stage A) and
+// then finish page j (stage B), whose partial was sent one iteration earlier.  P is
+// written (bf16) into the receive buffer the page arrived in and read from shared
+// memory by the PV MMA, which frees each S buffer as soon as it has been loaded, so
+// the MMA warp can compute scores two pages ahead.
 //
 // Roles (256 threads): warp 0 issues TMA loads, warp 1 allocates TMEM and issues
 // MMAs, warp 2 zeroes value rows past the sequence end before PV reads them,
-// warps 4..7 (one thread per head row = TMEM lane) stage q', exchange partial
-// scores, run the online softmax (log2 domain, lazy rescale by at most 2^8), write
-// P as bf16 into TMEM, rescale O when needed, and write the epilogue.
+// warp 3 recycles receive buffers (once a PV has consumed a buffer it re-arms it and
+// tells the peer it may send into it again), warps 4..7 (one thread per head row =
+// TMEM lane) stage q', exchange partial scores, run the online softmax (log2
+// domain, lazy rescale by at most 2^8), write P, rescale O when needed, and write
+// the epilogue.
 //
-// TMEM (512 columns): O [0,256) fp32, S double buffer [256,320) [320,384) fp32 with
-// P (bf16 pairs) aliased over the first 32 columns of its S buffer, q' latent half
-// [384,512) as bf16 pairs (the A operand of QK^T).
-// Shared memory: 3 stages x 5 boxes of [64 tokens x 64 dims] bf16 (128B swizzle):
-// boxes 0..3 = this CTA's latent dims (K-major B of QK^T and MN-major B of PV),
-// box 4 = the 64 rope dims (both CTAs load it; each uses its 32); the rope part of
-// q' [128 x 64] (A operand from shared memory); two 32 KB receive buffers for the
-// peer's partial scores.
+// TMEM (512 columns): O [0,256) fp32, S double buffer [256,320) [320,384) fp32,
+// q' latent half [384,512) as bf16 pairs (the A operand of the latent QK^T).
+// Shared memory: 3 stages x (4 latent boxes [64 tokens x 64 dims], 128B swizzle:
+// K-major B of QK^T and MN-major B of PV; 1 rope box [64 tokens x 32 dims], 64B
+// swizzle); this CTA's rope part of q' [128 x 32] (64B swizzle, A operand); one
+// 32 KB send buffer; two 32 KB receive buffers (partial scores in, then P).
 //
 // Every mbarrier wait is bounded by a time limit; on expiry the kernel records
-// MLA_ERR_DEVICE_TIMEOUT, tells the peer CTA to stop, drains its own TMA and MMA
-// work, frees TMEM and returns.  No trap.
+// MLA_ERR_DEVICE_TIMEOUT, tells the peer CTA to stop, drains its own TMA, bulk-copy
+// and MMA work, frees TMEM and returns.  No trap.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -46,28 +54,42 @@ using namespace sm100;
 
 constexpr int kThreads = 256;
 constexpr int kStages = 3;
-constexpr int kBoxBytes = 64 * 128;              // [64 rows x 64 bf16], 128B swizzle
-constexpr int kStageBytes = 5 * kBoxBytes;       // 40960
-constexpr int kQRopeBytes = 128 * 128;           // [128 heads x 64 rope dims]
-constexpr int kRxBytes = 128 * 64 * 4;           // [128 heads x 64 fp32]
-constexpr int kSmemStages = 0;
-constexpr int kSmemQRope = kStages * kStageBytes;            // 122880
-constexpr int kSmemRx = kSmemQRope + kQRopeBytes;             // 139264
-constexpr int kSmemBytes = kSmemRx + 2 * kRxBytes;            // 204800
+constexpr int kLatBox = 64 * 128;                 // [64 rows x 64 bf16], 128B swizzle
+constexpr int kRopeBox = 64 * 64;                 // [64 rows x 32 bf16], 64B swizzle
+constexpr int kStageBytes = 4 * kLatBox + kRopeBox;  // 36864
+constexpr int kXBytes = 128 * 64 * 4;             // [128 heads x 64 tokens] fp32 partial scores
+constexpr int kSmemQRope = kStages * kStageBytes;             // 110592
+constexpr int kSmemTx = kSmemQRope + 128 * 64;                // 118784
+constexpr int kSmemRx = kSmemTx + kXBytes;                    // 151552
+constexpr int kSmemBytes = kSmemRx + 2 * kXBytes;             // 217088
 constexpr int kSmemAlloc = kSmemBytes + 1024;                 // + alignment slack
 
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColO = 0, kColS = 256, kColQ = 384;
 
-constexpr uint32_t kIdescQK = idesc_bf16_f32(128, 64, 0, 0);   // A tmem/smem K-major, B K-major
-constexpr uint32_t kIdescPV = idesc_bf16_f32(128, 256, 0, 1);  // A tmem K-major, B MN-major
+constexpr uint32_t kIdescQK = idesc_bf16_f32(128, 64, 0, 0);   // A K-major (TMEM or smem), B K-major
+constexpr uint32_t kIdescPV = idesc_bf16_f32(128, 256, 0, 1);  // A (P, smem) K-major, B MN-major
 
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: P may reach 2^8 before O is rescaled
 
 enum Bar {
-  kKvFull = 0, kKvEmpty = kKvFull + kStages, kVReady = kKvEmpty + kStages, kSFull = kVReady + kStages,
-  kPFull = kSFull + 2, kRxFull = kPFull + 2, kTxFree = kRxFull + 2, kODone = kTxFree + 2, kOFull = kODone + 4,
-  kQReady = kOFull + 1, kDrain = kQReady + 1, kNumBars = kDrain + 1
+  kKvFull = 0,
+  kKvEmpty = kKvFull + kStages,
+  kVReady = kKvEmpty + kStages,
+  kSFull = kVReady + kStages,
+  kSFree = kSFull + 2,
+  kPFull = kSFree + 2,
+  kPvDone = kPFull + 2,
+  kRxFull = kPvDone + 2,
+  kPeerFree = kRxFull + 2,
+  kTxWritable = kPeerFree + 2,
+  kTxReady = kTxWritable + 1,
+  kRxRead = kTxReady + 1,
+  kODone = kRxRead + 1,  // [warp q][PV parity]: 8 barriers
+  kOFull = kODone + 8,
+  kQReady = kOFull + 1,
+  kDrain = kQReady + 1,
+  kNumBars = kDrain + 1
 };
 
 struct Piece {
@@ -127,12 +149,21 @@ __device__ __noinline__ bool wait_bar(uint32_t bar, uint32_t parity, const Ctl& 
   }
 }
 
+// Spin (bounded by time, ignoring the abort flag) until a phase completes: used only
+// while draining work that is already in flight.
+__device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, uint64_t limit_ns) {
+  const uint64_t t0 = now_ns();
+  while (!mbar_try_wait(bar, parity) && now_ns() - t0 < limit_ns) {
+  }
+}
+
 __device__ __forceinline__ int page_of(const DecodeArgs& a, int b, int p) {
   return a.block_table ? a.block_table[(size_t)b * a.max_blocks + p] : b * a.max_blocks + p;
 }
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
-    decode_tc_kernel(const __grid_constant__ CUtensorMap kv_map, const DecodeArgs a, uint64_t limit_ns) {
+    decode_tc_kernel(const __grid_constant__ CUtensorMap kv_map, const __grid_constant__ CUtensorMap rope_map,
+                     const DecodeArgs a, uint64_t limit_ns) {
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t bars[kNumBars];
   __shared__ uint32_t tmem_base_s;
@@ -140,7 +171,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
-  const uint32_t s_stage0 = sbase + kSmemStages, s_qrope = sbase + kSmemQRope, s_rx = sbase + kSmemRx;
+  const uint32_t s_qrope = sbase + kSmemQRope, s_tx = sbase + kSmemTx, s_rx = sbase + kSmemRx;
   auto bar = [&](int i) { return smem_u32(&bars[i]); };
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -159,17 +190,26 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       mbar_init(bar(kVReady + s), 1);
     }
     for (int u = 0; u < 2; ++u) {
-      mbar_init(bar(kSFull + u), 1);
-      mbar_init(bar(kPFull + u), 128);
-      mbar_init(bar(kRxFull + u), 128);
-      mbar_init(bar(kTxFree + u), 128);
+      mbar_init(bar(kSFull + u), 1);      // MMA commit
+      mbar_init(bar(kSFree + u), 128);    // every softmax thread has loaded S
+      mbar_init(bar(kPFull + u), 4);      // one arrival per softmax warp
+      mbar_init(bar(kPvDone + u), 1);     // MMA commit
+      mbar_init(bar(kRxFull + u), 1);     // armed (expect_tx) here, bytes from the peer
+      mbar_init(bar(kPeerFree + u), 1);   // the peer's recycler: its receive buffer is free and armed
     }
-    for (int q = 0; q < 4; ++q) mbar_init(bar(kODone + q), 1);
+    mbar_init(bar(kTxWritable), 1);
+    mbar_init(bar(kTxReady), 4);
+    mbar_init(bar(kRxRead), 4);
+    for (int q = 0; q < 8; ++q) mbar_init(bar(kODone + q), 1);
     mbar_init(bar(kOFull), 1);
     mbar_init(bar(kQReady), 128);
     mbar_init(bar(kDrain), 1);
+    // The first round of both receive buffers is armed before the peer may send.
+    mbar_expect_tx(bar(kRxFull + 0), kXBytes);
+    mbar_expect_tx(bar(kRxFull + 1), kXBytes);
     fence_mbar_init();
     tma_prefetch_desc(&kv_map);
+    tma_prefetch_desc(&rope_map);
   }
   if (warp == 1) {
     tmem_alloc(smem_u32(&tmem_base_s), kTmemCols);
@@ -196,22 +236,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           int pid = page_of(a, pc.b, p);
           if ((unsigned)pid >= (unsigned)np) pid = 0;  // reported by the softmax warps; load something valid
           if (a.withhold_arrive && w == 0 && rank == 0 && it == 1) continue;  // timeout test: never arrives
-          const uint32_t dst = s_stage0 + s * kStageBytes;
+          const uint32_t dst = sbase + s * kStageBytes;
           mbar_expect_tx(bar(kKvFull + s), kStageBytes);
           const int y = pid * kPage;
 #pragma unroll
-          for (int i = 0; i < 4; ++i) tma_load_2d(dst + i * kBoxBytes, &kv_map, 256 * rank + 64 * i, y, bar(kKvFull + s));
-          tma_load_2d(dst + 4 * kBoxBytes, &kv_map, kDLatent, y, bar(kKvFull + s));
+          for (int i = 0; i < 4; ++i) tma_load_2d(dst + i * kLatBox, &kv_map, 256 * rank + 64 * i, y, bar(kKvFull + s));
+          tma_load_2d(dst + 4 * kLatBox, &rope_map, kDLatent + 32 * rank, y, bar(kKvFull + s));
         }
       }
       // Drain: every load issued into a stage lands before the CTA may exit (bounded).
       for (int k = 0; k < kStages && k < it; ++k) {
         const int j = it - 1 - k;
         if (a.withhold_arrive && w == 0 && rank == 0 && j == 1) continue;
-        const int s = j % kStages;
-        const uint64_t t0 = now_ns();
-        while (!mbar_try_wait(bar(kKvFull + s), (j / kStages) & 1) && now_ns() - t0 < limit_ns) {
-        }
+        drain_wait(bar(kKvFull + j % kStages), (j / kStages) & 1, limit_ns);
       }
     }
     __syncwarp();
@@ -222,56 +259,59 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       Piece pc;
       int it = 0, piece = 0;
       bool ok = true;
-      auto issue_pv = [&](int itp, bool first) -> bool {
-        const int s = itp % kStages, u = itp & 1;
-        if (!wait_bar(bar(kPFull + u), (itp >> 1) & 1, ctl)) return false;
-        if (!wait_bar(bar(kVReady + s), (itp / kStages) & 1, ctl)) return false;
+      auto issue_qk = [&](int g) -> bool {
+        const int s = g % kStages, u = g & 1;
+        if (g >= 2 && !wait_bar(bar(kSFree + u), ((g - 2) >> 1) & 1, ctl)) return false;
+        if (!wait_bar(bar(kKvFull + s), (g / kStages) & 1, ctl)) return false;
         tc_fence_after();
-        const uint32_t vbase = s_stage0 + s * kStageBytes;
-        const uint32_t p_col = tmem + kColS + 64 * u;
+        const uint32_t kbase = sbase + s * kStageBytes;
+        const uint32_t d = tmem + kColS + 64 * u;
+#pragma unroll
+        for (int kc = 0; kc < 16; ++kc)
+          mma_ts(d, tmem + kColQ + kc * 8, desc_sw128(kbase + (kc >> 2) * kLatBox + (kc & 3) * 32, 16, 1024),
+                 kIdescQK, kc > 0 ? 1u : 0u);
+#pragma unroll
+        for (int i = 0; i < 2; ++i)
+          mma_ss(d, desc_sw64(s_qrope + i * 32, 16, 512), desc_sw64(kbase + 4 * kLatBox + i * 32, 16, 512), kIdescQK,
+                 1u);
+        mma_commit(bar(kSFull + u));
+        return true;
+      };
+      auto issue_pv = [&](int g, bool first) -> bool {
+        const int s = g % kStages, u = g & 1;
+        if (!wait_bar(bar(kPFull + u), (g >> 1) & 1, ctl)) return false;
+        if (!wait_bar(bar(kVReady + s), (g / kStages) & 1, ctl)) return false;
+        tc_fence_after();
+        const uint32_t vbase = sbase + s * kStageBytes;
+        const uint32_t pbase = s_rx + u * kXBytes;
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
-          mma_ts(tmem + kColO, p_col + kk * 8, desc_sw128(vbase + kk * 2048, 8192, 1024), kIdescPV,
-                 (first && kk == 0) ? 0u : 1u);
+          mma_ss(tmem + kColO, desc_sw128(pbase + kk * 32, 16, 1024), desc_sw128(vbase + kk * 2048, 8192, 1024),
+                 kIdescPV, (first && kk == 0) ? 0u : 1u);
         mma_commit(bar(kKvEmpty + s));
+        mma_commit(bar(kPvDone + u));
+        // PV(g) is tracked on the barriers of its parity: the next completion there
+        // is PV(g+2), which needs P(g+2), so a waiter is never two phases behind.
 #pragma unroll
-        for (int q = 0; q < 4; ++q) mma_commit(bar(kODone + q));
+        for (int q = 0; q < 4; ++q) mma_commit(bar(kODone + 2 * q + u));
         return true;
       };
       while (ok && pi.next(pc)) {
         if (!wait_bar(bar(kQReady), piece & 1, ctl)) { ok = false; break; }
         tc_fence_after();
         const int n = pc.pe - pc.pa;
+        ok = issue_qk(it) && (n < 2 || issue_qk(it + 1));
         for (int j = 0; j < n && ok; ++j) {
-          const int itj = it + j, s = itj % kStages, u = itj & 1;
-          if (!wait_bar(bar(kKvFull + s), (itj / kStages) & 1, ctl)) { ok = false; break; }
-          tc_fence_after();
-          const uint32_t kbase = s_stage0 + s * kStageBytes;
-          const uint32_t d = tmem + kColS + 64 * u;
-#pragma unroll
-          for (int kc = 0; kc < 16; ++kc)
-            mma_ts(d, tmem + kColQ + kc * 8, desc_sw128(kbase + (kc >> 2) * kBoxBytes + (kc & 3) * 32, 16, 1024),
-                   kIdescQK, kc > 0 ? 1u : 0u);
-#pragma unroll
-          for (int i = 0; i < 2; ++i) {
-            const int kr = 2 * (int)rank + i;
-            mma_ss(d, desc_sw128(s_qrope + kr * 32, 16, 1024),
-                   desc_sw128(kbase + 4 * kBoxBytes + kr * 32, 16, 1024), kIdescQK, 1u);
-          }
-          mma_commit(bar(kSFull + u));
-          if (j > 0 && !issue_pv(itj - 1, j == 1)) { ok = false; break; }
+          ok = issue_pv(it + j, j == 0) && (j + 2 >= n || issue_qk(it + j + 2));
         }
         if (!ok) break;
-        if (!issue_pv(it + n - 1, n == 1)) { ok = false; break; }
         mma_commit(bar(kOFull));
         it += n;
         ++piece;
       }
       // Drain every MMA this thread issued before TMEM is released.
       mma_commit(bar(kDrain));
-      const uint64_t t0 = now_ns();
-      while (!mbar_try_wait(bar(kDrain), 0) && now_ns() - t0 < limit_ns) {
-      }
+      drain_wait(bar(kDrain), 0, limit_ns);
     }
     __syncwarp();
   } else if (warp == 2) {
@@ -289,12 +329,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         if (valid < kPage) {
           // Rows >= valid may hold anything (NaN included); P is 0 there but 0 * NaN is
           // NaN, so zero them in the four value boxes before PV reads the stage.
-          uint8_t* st = smem + kSmemStages + s * kStageBytes;
+          uint8_t* st = smem + s * kStageBytes;
           const int nrow = kPage - valid;
           for (int idx = lane; idx < nrow * 4 * 8; idx += 32) {
             const int box = idx / (nrow * 8), rem = idx % (nrow * 8);
             const int row = valid + rem / 8, chunk = rem % 8;
-            *reinterpret_cast<uint4*>(st + box * kBoxBytes + row * 128 + chunk * 16) = make_uint4(0, 0, 0, 0);
+            *reinterpret_cast<uint4*>(st + box * kLatBox + row * 128 + chunk * 16) = make_uint4(0, 0, 0, 0);
           }
           fence_proxy_async();
         }
@@ -302,25 +342,89 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         if (lane == 0) mbar_arrive(bar(kVReady + s));
       }
     }
-  } else if (warp >= 4) {
+  } else if (warp == 3) {
+    // ------------------------------------------------------------ receive-buffer recycler
+    // After the PV of page g has consumed receive buffer g&1 (which held the peer's
+    // partial and then P), arm it for page g+2 and let the peer send into it.
+    if (lane == 0) {
+      PieceIter pi(sc, w);
+      Piece pc;
+      int g = 0;
+      bool ok = true;
+      const uint32_t peer_free = map_to_rank(bar(kPeerFree), peer);
+      while (ok && pi.next(pc)) {
+        for (int p = pc.pa; p < pc.pe; ++p, ++g) {
+          const int u = g & 1;
+          if (!wait_bar(bar(kPvDone + u), (g >> 1) & 1, ctl)) { ok = false; break; }
+          mbar_expect_tx(bar(kRxFull + u), kXBytes);
+          mbar_arrive_cluster(peer_free + u * 8);
+        }
+      }
+    }
+    __syncwarp();
+  } else {
     // ------------------------------------------------------------ softmax warpgroup
     const int row = tid - 128;             // head row = TMEM lane
     const int q = warp & 3;                // lane quadrant of this warp
     const uint32_t lane_off = (uint32_t)(32 * q) << 16;
     const uint32_t t_o = tmem + lane_off + kColO;
     const uint32_t t_q = tmem + lane_off + kColQ;
-    const uint32_t rx_peer = map_to_rank(s_rx, peer) + row * 256;
+    const uint32_t rx_peer = map_to_rank(s_rx, peer);
     const uint32_t peer_rx_full = map_to_rank(bar(kRxFull), peer);
-    const uint32_t peer_tx_free = map_to_rank(bar(kTxFree), peer);
+    const bool sender = row == 0;
     const float scale2 = a.scale * kLog2e;
+    uint8_t* txrow = smem + kSmemTx + row * 256;
     PieceIter pi(sc, w);
     Piece pc;
-    int it = 0, piece = 0, od = 0;  // od: o_done phases known complete
+    int it = 0, piece = 0;
     bool ok = true;
+    float own0[64], own1[64];
+
+    // Stage A of global page g: load this CTA's partial scores, free the S buffer,
+    // scale to log2 units, and send them to the peer.
+    auto stage_a = [&](int g, float (&own)[64]) -> bool {
+      const int u = g & 1, k = g >> 1;
+      if (!__all_sync(0xffffffffu, wait_bar(bar(kSFull + u), k & 1, ctl))) return false;
+      tc_fence_after();
+      {
+        uint32_t r0[32], r1[32];
+        tmem_ld32(tmem + lane_off + kColS + 64 * u, r0);
+        tmem_ld32(tmem + lane_off + kColS + 64 * u + 32, r1);
+        tmem_wait_ld();
+#pragma unroll
+        for (int c = 0; c < 32; ++c) {
+          own[c] = __uint_as_float(r0[c]) * scale2;
+          own[32 + c] = __uint_as_float(r1[c]) * scale2;
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(bar(kSFree + u));
+      // The previous page's copy out of the send buffer must have finished reading it.
+      if (sender) {
+        bulk_wait_read_all();
+        mbar_arrive(bar(kTxWritable));
+      }
+      if (!__all_sync(0xffffffffu, wait_bar(bar(kTxWritable), g & 1, ctl))) return false;
+#pragma unroll
+      for (int c = 0; c < 16; ++c)
+        *reinterpret_cast<float4*>(txrow + ((c ^ (row & 7)) * 16)) =
+            make_float4(own[4 * c], own[4 * c + 1], own[4 * c + 2], own[4 * c + 3]);
+      fence_proxy_async();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(kTxReady));
+      bool good = true;
+      if (sender) {
+        // Our rows are written, and the peer has freed and armed its receive buffer u.
+        good = wait_bar(bar(kPeerFree + u), (k & 1) ^ 1, ctl) && wait_bar(bar(kTxReady), g & 1, ctl);
+        if (good) bulk_copy_to_peer(rx_peer + u * kXBytes, s_tx, kXBytes, peer_rx_full + u * 8);
+      }
+      return __all_sync(0xffffffffu, good);
+    };
+
     while (ok && pi.next(pc)) {
       const int b = pc.b, n = pc.pe - pc.pa;
       const int T = a.seqlens[b];
-      // ---- stage q' for this sequence: latent half -> TMEM, rope -> smem (128B swizzle)
+      // ---- stage q' for this sequence: latent half -> TMEM, this CTA's 32 rope dims -> smem
       {
         uint32_t qv[16];
         const bool live = row < a.heads;
@@ -337,11 +441,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           }
           tmem_st16(t_q + c * 16, qv);
         }
-        uint8_t* qr = smem + kSmemQRope + row * 128;
+        uint8_t* qr = smem + kSmemQRope + row * 64;
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          const uint4 v = live ? src[kDLatent / 8 + c] : make_uint4(0, 0, 0, 0);
-          *reinterpret_cast<uint4*>(qr + ((c ^ (row & 7)) * 16)) = v;
+        for (int c = 0; c < 4; ++c) {  // 64B swizzle: 16-byte chunk c of row r at c ^ ((r >> 1) & 3)
+          const uint4 v = live ? src[kDLatent / 8 + 4 * rank + c] : make_uint4(0, 0, 0, 0);
+          *reinterpret_cast<uint4*>(qr + ((c ^ ((row >> 1) & 3)) * 16)) = v;
         }
         tmem_wait_st();
         fence_proxy_async();
@@ -350,121 +454,103 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       }
       float m = -INFINITY, l = 0.f;
       bool bad = false;
-      for (int j = 0; j < n; ++j) {
-        const int itj = it + j, u = itj & 1, ph = (itj >> 1) & 1, p = pc.pa + j;
-        if (!__all_sync(0xffffffffu, wait_bar(bar(kSFull + u), ph, ctl))) { ok = false; break; }
-        tc_fence_after();
-        // PV(j-2) finished before QK^T(j) did: retire its o_done phase (no stall).
-        while (od <= it + j - 2) {
-          if (!__all_sync(0xffffffffu, wait_bar(bar(kODone + q), od & 1, ctl))) { ok = false; break; }
-          ++od;
-        }
-        if (!ok) break;
-        float x[64];
-        {
-          uint32_t r0[32], r1[32];
-          tmem_ld32(tmem + lane_off + kColS + 64 * u, r0);
-          tmem_ld32(tmem + lane_off + kColS + 64 * u + 32, r1);
-          tmem_wait_ld();
+      int pid_next = page_of(a, b, pc.pa);
+      ok = (it & 1) ? stage_a(it, own1) : stage_a(it, own0);
+      // Stage B of page j of this piece: add the peer's partial, online softmax, write P.
+      auto stage_b = [&](int j, float (&x)[64]) -> bool {
+        const int g = it + j, u = g & 1, k = g >> 1, p = pc.pa + j;
+          if (!__all_sync(0xffffffffu, wait_bar(bar(kRxFull + u), k & 1, ctl))) return false;
+          {
+            const uint8_t* rxrow = smem + kSmemRx + u * kXBytes + row * 256;
 #pragma unroll
-          for (int k = 0; k < 32; ++k) {
-            x[k] = __uint_as_float(r0[k]);
-            x[32 + k] = __uint_as_float(r1[k]);
-          }
-        }
-        // ---- exchange partial scores with the peer CTA
-        if (!__all_sync(0xffffffffu, wait_bar(bar(kTxFree + u), ph ^ 1, ctl))) { ok = false; break; }
-        const uint32_t dst = rx_peer + u * kRxBytes;
-#pragma unroll
-        for (int c = 0; c < 16; ++c)
-          st_cluster_v4(dst + ((c ^ (row & 7)) * 16), x[4 * c], x[4 * c + 1], x[4 * c + 2], x[4 * c + 3]);
-        mbar_arrive_cluster(peer_rx_full + u * 8);
-        if (!__all_sync(0xffffffffu, wait_bar(bar(kRxFull + u), ph, ctl))) { ok = false; break; }
-        {
-          const uint8_t* src = smem + kSmemRx + u * kRxBytes + row * 256;
-#pragma unroll
-          for (int c = 0; c < 16; ++c) {
-            const float4 v = *reinterpret_cast<const float4*>(src + ((c ^ (row & 7)) * 16));
-            // Both CTAs add (own + peer) for their own first operand; fp32 addition is
-            // commutative, so both hold bit-identical scores.
-            x[4 * c + 0] += v.x;
-            x[4 * c + 1] += v.y;
-            x[4 * c + 2] += v.z;
-            x[4 * c + 3] += v.w;
-          }
-        }
-        mbar_arrive_cluster(peer_tx_free + u * 8);
-        // ---- online softmax, log2 domain
-        const int pid = page_of(a, b, p);
-        if ((unsigned)pid >= (unsigned)np) {
-          bad = true;
-          set_device_error(a.err, MLA_ERR_DEVICE_BAD_PAGE);
-        }
-        const int valid = min(kPage, T - p * kPage);
-        float tmax = -INFINITY;
-#pragma unroll
-        for (int k = 0; k < 64; ++k) {
-          x[k] = k < valid ? x[k] * scale2 : -INFINITY;
-          tmax = fmaxf(tmax, x[k]);
-        }
-        const float m_new = fmaxf(m, tmax);
-        const bool need = m_new > m + kRescaleThreshold;
-        const float alpha = need ? fast_exp2(m - m_new) : 1.f;
-        if (need) m = m_new;
-        if (__any_sync(0xffffffffu, need && j > 0)) {
-          // O must hold PV(j-1) before it is rescaled (rare path).
-          while (od <= it + j - 1) {
-            if (!__all_sync(0xffffffffu, wait_bar(bar(kODone + q), od & 1, ctl))) { ok = false; break; }
-            ++od;
-          }
-          if (!ok) break;
-          tc_fence_after();
-#pragma unroll 1
-          for (int c = 0; c < 8; ++c) {
-            uint32_t r[32];
-            tmem_ld32(t_o + c * 32, r);
-            tmem_wait_ld();
-            uint32_t w0[16], w1[16];
-#pragma unroll
-            for (int k = 0; k < 16; ++k) {
-              w0[k] = __float_as_uint(__uint_as_float(r[k]) * alpha);
-              w1[k] = __float_as_uint(__uint_as_float(r[16 + k]) * alpha);
+            for (int c = 0; c < 16; ++c) {
+              const float4 v = *reinterpret_cast<const float4*>(rxrow + ((c ^ (row & 7)) * 16));
+              // fp32 addition is commutative: both CTAs hold the same sums.
+              x[4 * c + 0] += v.x;
+              x[4 * c + 1] += v.y;
+              x[4 * c + 2] += v.z;
+              x[4 * c + 3] += v.w;
             }
-            tmem_st16(t_o + c * 32, w0);
-            tmem_st16(t_o + c * 32 + 16, w1);
           }
-          tmem_wait_st();
-        }
-        l *= alpha;
-        uint32_t pk[32];
-        float rs = 0.f;
-#pragma unroll
-        for (int k = 0; k < 32; ++k) {
-          const float p0 = fast_exp2(x[2 * k] - m);
-          const float p1 = fast_exp2(x[2 * k + 1] - m);
-          rs += p0 + p1;
-          pk[k] = pack_bf16x2(p0, p1);
-        }
-        l += rs;
-        {
-          uint32_t h0[16], h1[16];
-#pragma unroll
-          for (int k = 0; k < 16; ++k) {
-            h0[k] = pk[k];
-            h1[k] = pk[16 + k];
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bar(kRxRead));
+          const int pid = pid_next;
+          if (j + 1 < n) pid_next = page_of(a, b, p + 1);  // used next page: latency off the chain
+          if ((unsigned)pid >= (unsigned)np) {
+            bad = true;
+            set_device_error(a.err, MLA_ERR_DEVICE_BAD_PAGE);
           }
-          tmem_st16(tmem + lane_off + kColS + 64 * u, h0);
-          tmem_st16(tmem + lane_off + kColS + 64 * u + 16, h1);
+          const int valid = min(kPage, T - p * kPage);
+          float tmax = -INFINITY;
+#pragma unroll
+          for (int c = 0; c < 64; ++c) {
+            x[c] = c < valid ? x[c] : -INFINITY;
+            tmax = fmaxf(tmax, x[c]);
+          }
+          const float m_new = fmaxf(m, tmax);
+          const bool need = m_new > m + kRescaleThreshold;
+          const float alpha = need ? fast_exp2(m - m_new) : 1.f;
+          if (need) m = m_new;
+          if (__any_sync(0xffffffffu, need && j > 0)) {
+            // O must hold PV(g-1) before it is rescaled (rare path).
+            const int x = g - 1;
+            if (!__all_sync(0xffffffffu, wait_bar(bar(kODone + 2 * q + (x & 1)), (x >> 1) & 1, ctl))) return false;
+            tc_fence_after();
+#pragma unroll 1
+            for (int c = 0; c < 8; ++c) {
+              uint32_t r[32];
+              tmem_ld32(t_o + c * 32, r);
+              tmem_wait_ld();
+              uint32_t w0[16], w1[16];
+#pragma unroll
+              for (int e = 0; e < 16; ++e) {
+                w0[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
+                w1[e] = __float_as_uint(__uint_as_float(r[16 + e]) * alpha);
+              }
+              tmem_st16(t_o + c * 32, w0);
+              tmem_st16(t_o + c * 32 + 16, w1);
+            }
+            tmem_wait_st();
+            tc_fence_before();
+          }
+          l *= alpha;
+          uint32_t pk[32];
+          float rs = 0.f;
+#pragma unroll
+          for (int c = 0; c < 32; ++c) {
+            const float p0 = fast_exp2(x[2 * c] - m);
+            const float p1 = fast_exp2(x[2 * c + 1] - m);
+            rs += p0 + p1;
+            pk[c] = pack_bf16x2(p0, p1);
+          }
+          l += rs;
+          // Every row of the receive buffer has been read: overwrite it with P
+          // ([128 heads x 64 tokens] bf16, K-major, 128B swizzle: the PV A operand).
+          if (!__all_sync(0xffffffffu, wait_bar(bar(kRxRead), g & 1, ctl))) return false;
+          {
+            uint8_t* prow = smem + kSmemRx + u * kXBytes + row * 128;
+#pragma unroll
+            for (int c = 0; c < 8; ++c)
+              *reinterpret_cast<uint4*>(prow + ((c ^ (row & 7)) * 16)) =
+                  make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+          }
+          fence_proxy_async();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bar(kPFull + u));
+        return true;
+      };
+      for (int j = 0; j < n && ok; ++j) {
+        const int g = it + j;
+        if (j + 1 < n) {
+          ok = (g & 1) ? stage_a(g + 1, own0) : stage_a(g + 1, own1);
+          if (!ok) break;
         }
-        tmem_wait_st();
-        tc_fence_before();
-        mbar_arrive(bar(kPFull + u));
+        ok = (g & 1) ? stage_b(j, own1) : stage_b(j, own0);
       }
       if (!ok) break;
       // ---- epilogue: O / l (this CTA's 256 dims), lse
       if (!__all_sync(0xffffffffu, wait_bar(bar(kOFull), piece & 1, ctl))) { ok = false; break; }
       tc_fence_after();
-      od = it + n;  // every PV of this piece has completed
       const float inv = bad ? NAN : 1.f / l;
       const float lse_v = bad ? NAN : (m + __log2f(l)) * kLn2;
       const bool complete = pc.pa == 0 && pc.pe == sc.seq_start[b + 1] - sc.seq_start[b];
@@ -486,9 +572,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         if (row < a.heads) {
           float4* dst = reinterpret_cast<float4*>(obase + (size_t)row * kDLatent + 256 * rank + 32 * c);
 #pragma unroll
-          for (int k = 0; k < 8; ++k)
-            dst[k] = make_float4(__uint_as_float(r[4 * k]) * inv, __uint_as_float(r[4 * k + 1]) * inv,
-                                 __uint_as_float(r[4 * k + 2]) * inv, __uint_as_float(r[4 * k + 3]) * inv);
+          for (int e = 0; e < 8; ++e)
+            dst[e] = make_float4(__uint_as_float(r[4 * e]) * inv, __uint_as_float(r[4 * e + 1]) * inv,
+                                 __uint_as_float(r[4 * e + 2]) * inv, __uint_as_float(r[4 * e + 3]) * inv);
         }
       }
       if (rank == 0 && row < a.heads) lbase[row] = lse_v;
@@ -496,6 +582,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       it += n;
       ++piece;
     }
+    if (sender) bulk_wait_all();  // our copies into the peer have landed
   }
 
   // ------------------------------------------------------------ teardown
@@ -550,18 +637,25 @@ cudaError_t launch_decode_tc(const DecodeArgs& a, cudaStream_t stream) {
   }
   auto encode = get_encode();
   if (!encode) return cudaErrorNotSupported;
-  CUtensorMap map;
+  // The cache as a 2-D tensor [rows, 576]: latent boxes of 64 dims (128B swizzle) and
+  // rope boxes of 32 dims (64B swizzle), 64 rows (one page) each.
+  CUtensorMap kv_map, rope_map;
   const uint64_t rows = (uint64_t)(a.block_table ? a.num_pages : a.batch * a.max_blocks) * kPage;
   cuuint64_t dims[2] = {(cuuint64_t)kDQK, (cuuint64_t)rows};
   cuuint64_t strides[1] = {(cuuint64_t)kDQK * 2};
-  cuuint32_t box[2] = {64, 64};
   cuuint32_t estr[2] = {1, 1};
-  CUresult r = encode(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<__nv_bfloat16*>(a.kv), dims, strides,
-                      box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+  cuuint32_t box_lat[2] = {64, 64};
+  cuuint32_t box_rope[2] = {32, 64};
+  CUresult r = encode(&kv_map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<__nv_bfloat16*>(a.kv), dims, strides,
+                      box_lat, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                       CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
+  r = encode(&rope_map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<__nv_bfloat16*>(a.kv), dims, strides,
+             box_rope, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
   const uint64_t limit_ns = (uint64_t)(a.wait_limit > 0 ? a.wait_limit : 1000) * 1000000ull;  // wait_limit in ms
-  decode_tc_kernel<<<2 * a.sched.num_workers, kThreads, kSmemAlloc, stream>>>(map, a, limit_ns);
+  decode_tc_kernel<<<2 * a.sched.num_workers, kThreads, kSmemAlloc, stream>>>(kv_map, rope_map, a, limit_ns);
   return cudaGetLastError();
 }
 
