@@ -9,31 +9,32 @@
 // it: CTA r keeps O[:, 256r : 256r+256) and contracts the scores over its own dims
 // (latent [256r, 256r+256) plus rope [512+32r, 512+32r+32)).  Each CTA therefore
 // loads only its part of every row (HBM and L2 traffic 1x), computes a partial S,
-// and the two fp32 partials are exchanged through distributed shared memory by bulk
-// copies (32 KB per page each way) and added in the same order on both sides, so
-// both CTAs run a bit-identical softmax.
+// and the two partials are exchanged through distributed shared memory by bulk
+// copies and added, so both CTAs run a bit-identical softmax.  Each exchanged score
+// is the fp32 value rounded to 24 bits (sign, exponent, 15 mantissa bits; relative
+// error <= 2^-16), 4 values in 12 bytes: 24 KB per page each way.
 //
 // Pipeline.  The exchange has a long latency, so the softmax threads are software
 // pipelined: in each iteration they first send page j+1's partial (stage A) and
-// then finish page j (stage B), whose partial was sent one iteration earlier.  P is
-// written (bf16) into the receive buffer the page arrived in and read from shared
-// memory by the PV MMA, which frees each S buffer as soon as it has been loaded, so
-// the MMA warp can compute scores two pages ahead.
+// then finish page j (stage B), whose partial was sent one iteration earlier.  A
+// receive buffer is handed back to the peer as soon as it has been read.  P is
+// written (bf16) to shared memory and read from there by the PV MMA, which frees
+// each S buffer as soon as it has been loaded, so score MMAs run ahead.
 //
-// Roles (256 threads): warp 0 issues TMA loads, warp 1 allocates TMEM and issues
-// MMAs, warp 2 zeroes value rows past the sequence end before PV reads them,
-// warp 3 recycles receive buffers (once a PV has consumed a buffer it re-arms it and
-// tells the peer it may send into it again), warps 4..7 (one thread per head row =
-// TMEM lane) stage q', exchange partial scores, run the online softmax (log2
-// domain, lazy rescale by at most 2^8), write P, rescale O when needed, and write
-// the epilogue.
+// Roles (384 threads): warp 0 issues TMA loads, warp 1 allocates TMEM and issues
+// MMAs (whichever of the next score MMA and the next PV is ready first), warp 2
+// zeroes value rows past the sequence end before PV reads them, warp 3 idles,
+// warps 4..11 are two softmax warpgroups (one thread per
+// head row = TMEM lane, each warpgroup half of every page's columns) that stage q',
+// exchange partial scores, run the online softmax (log2 domain, lazy rescale by at
+// most 2^8), write P, rescale O when needed, and write the epilogue.
 //
 // TMEM (512 columns): O [0,256) fp32, S double buffer [256,320) [320,384) fp32,
 // q' latent half [384,512) as bf16 pairs (the A operand of the latent QK^T).
 // Shared memory: 3 stages x (4 latent boxes [64 tokens x 64 dims], 128B swizzle:
 // K-major B of QK^T and MN-major B of PV; 1 rope box [64 tokens x 32 dims], 64B
 // swizzle); this CTA's rope part of q' [128 x 32] (64B swizzle, A operand); one
-// 32 KB send buffer; two 32 KB receive buffers (partial scores in, then P).
+// 24 KB send buffer; two 24 KB receive buffers; two 16 KB P buffers (128B swizzle).
 //
 // Every mbarrier wait is bounded by a time limit; on expiry the kernel records
 // MLA_ERR_DEVICE_TIMEOUT, tells the peer CTA to stop, drains its own TMA, bulk-copy
@@ -52,16 +53,21 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kThreads = 256;
+constexpr int kThreads = 384;
 constexpr int kStages = 3;
 constexpr int kLatBox = 64 * 128;                 // [64 rows x 64 bf16], 128B swizzle
 constexpr int kRopeBox = 64 * 64;                 // [64 rows x 32 bf16], 64B swizzle
 constexpr int kStageBytes = 4 * kLatBox + kRopeBox;  // 36864
-constexpr int kXBytes = 128 * 64 * 4;             // [128 heads x 64 tokens] fp32 partial scores
+constexpr int kXRow = 64 * 3;                     // one head row of partial scores, 24 bits per value
+constexpr int kXBytes = 128 * kXRow;              // 24576: [128 heads x 64 tokens] partial scores
+constexpr int kPBytes = 128 * 128;                // [128 heads x 64 tokens] bf16 P
 constexpr int kSmemQRope = kStages * kStageBytes;             // 110592
 constexpr int kSmemTx = kSmemQRope + 128 * 64;                // 118784
-constexpr int kSmemRx = kSmemTx + kXBytes;                    // 151552
-constexpr int kSmemBytes = kSmemRx + 2 * kXBytes;             // 217088
+constexpr int kSmemRx = kSmemTx + kXBytes;                    // 143360: 2 receive buffers
+constexpr int kSmemP = kSmemRx + 2 * kXBytes;                 // 192512: 2 P buffers (1024-aligned)
+constexpr int kSmemHmax = kSmemP + 2 * kPBytes;               // 225280: half-row maxima [2][2][128]
+constexpr int kSmemLsum = kSmemHmax + 2 * 2 * 128 * 4;        // 227328: half-row sums [2][128]
+constexpr int kSmemBytes = kSmemLsum + 2 * 128 * 4;           // 228352
 constexpr int kSmemAlloc = kSmemBytes + 1024;                 // + alignment slack
 
 constexpr uint32_t kTmemCols = 512;
@@ -79,14 +85,14 @@ enum Bar {
   kSFull = kVReady + kStages,
   kSFree = kSFull + 2,
   kPFull = kSFree + 2,
-  kPvDone = kPFull + 2,
-  kRxFull = kPvDone + 2,
+  kRxFull = kPFull + 2,
   kPeerFree = kRxFull + 2,
   kTxWritable = kPeerFree + 2,
   kTxReady = kTxWritable + 1,
-  kRxRead = kTxReady + 1,
-  kODone = kRxRead + 1,  // [warp q][PV parity]: 8 barriers
-  kOFull = kODone + 8,
+  kXMax = kTxReady + 1,   // half-row maxima published (and the receive buffer fully read)
+  kLSync = kXMax + 1,     // half-row sums published (epilogue)
+  kODone = kLSync + 1,    // [softmax warp][PV parity]: 16 barriers
+  kOFull = kODone + 16,
   kQReady = kOFull + 1,
   kDrain = kQReady + 1,
   kNumBars = kDrain + 1
@@ -171,7 +177,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
-  const uint32_t s_qrope = sbase + kSmemQRope, s_tx = sbase + kSmemTx, s_rx = sbase + kSmemRx;
+  const uint32_t s_qrope = sbase + kSmemQRope, s_tx = sbase + kSmemTx, s_rx = sbase + kSmemRx, s_p = sbase + kSmemP;
   auto bar = [&](int i) { return smem_u32(&bars[i]); };
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -191,18 +197,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     }
     for (int u = 0; u < 2; ++u) {
       mbar_init(bar(kSFull + u), 1);      // MMA commit
-      mbar_init(bar(kSFree + u), 128);    // every softmax thread has loaded S
-      mbar_init(bar(kPFull + u), 4);      // one arrival per softmax warp
-      mbar_init(bar(kPvDone + u), 1);     // MMA commit
+      mbar_init(bar(kSFree + u), 256);    // every softmax thread has loaded its half of S
+      mbar_init(bar(kPFull + u), 8);      // one arrival per softmax warp
       mbar_init(bar(kRxFull + u), 1);     // armed (expect_tx) here, bytes from the peer
-      mbar_init(bar(kPeerFree + u), 1);   // the peer's recycler: its receive buffer is free and armed
+      mbar_init(bar(kPeerFree + u), 1);   // the peer's receive buffer u is read and re-armed
     }
     mbar_init(bar(kTxWritable), 1);
-    mbar_init(bar(kTxReady), 4);
-    mbar_init(bar(kRxRead), 4);
-    for (int q = 0; q < 8; ++q) mbar_init(bar(kODone + q), 1);
+    mbar_init(bar(kTxReady), 8);
+    mbar_init(bar(kXMax), 8);
+    mbar_init(bar(kLSync), 8);
+    for (int q = 0; q < 16; ++q) mbar_init(bar(kODone + q), 1);
     mbar_init(bar(kOFull), 1);
-    mbar_init(bar(kQReady), 128);
+    mbar_init(bar(kQReady), 256);
     mbar_init(bar(kDrain), 1);
     // The first round of both receive buffers is armed before the peer may send.
     mbar_expect_tx(bar(kRxFull + 0), kXBytes);
@@ -259,10 +265,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       Piece pc;
       int it = 0, piece = 0;
       bool ok = true;
-      auto issue_qk = [&](int g) -> bool {
+      // Issues whichever is ready first: the next score MMA (its S buffer freed and its
+      // page loaded) or the next PV (its P written and its value rows cleaned), so score
+      // MMAs never queue behind a PV that waits for the softmax.
+      auto do_qk = [&](int g) {
         const int s = g % kStages, u = g & 1;
-        if (g >= 2 && !wait_bar(bar(kSFree + u), ((g - 2) >> 1) & 1, ctl)) return false;
-        if (!wait_bar(bar(kKvFull + s), (g / kStages) & 1, ctl)) return false;
         tc_fence_after();
         const uint32_t kbase = sbase + s * kStageBytes;
         const uint32_t d = tmem + kColS + 64 * u;
@@ -275,34 +282,61 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           mma_ss(d, desc_sw64(s_qrope + i * 32, 16, 512), desc_sw64(kbase + 4 * kLatBox + i * 32, 16, 512), kIdescQK,
                  1u);
         mma_commit(bar(kSFull + u));
-        return true;
       };
-      auto issue_pv = [&](int g, bool first) -> bool {
+      auto do_pv = [&](int g, bool first) {
         const int s = g % kStages, u = g & 1;
-        if (!wait_bar(bar(kPFull + u), (g >> 1) & 1, ctl)) return false;
-        if (!wait_bar(bar(kVReady + s), (g / kStages) & 1, ctl)) return false;
         tc_fence_after();
         const uint32_t vbase = sbase + s * kStageBytes;
-        const uint32_t pbase = s_rx + u * kXBytes;
+        const uint32_t pbase = s_p + u * kPBytes;
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
           mma_ss(tmem + kColO, desc_sw128(pbase + kk * 32, 16, 1024), desc_sw128(vbase + kk * 2048, 8192, 1024),
                  kIdescPV, (first && kk == 0) ? 0u : 1u);
         mma_commit(bar(kKvEmpty + s));
-        mma_commit(bar(kPvDone + u));
         // PV(g) is tracked on the barriers of its parity: the next completion there
         // is PV(g+2), which needs P(g+2), so a waiter is never two phases behind.
 #pragma unroll
-        for (int q = 0; q < 4; ++q) mma_commit(bar(kODone + 2 * q + u));
-        return true;
+        for (int q = 0; q < 8; ++q) mma_commit(bar(kODone + 2 * q + u));
+      };
+      auto qk_ready = [&](int g) {
+        return (g < 2 || mbar_test(bar(kSFree + (g & 1)), ((g - 2) >> 1) & 1)) &&
+               mbar_test(bar(kKvFull + g % kStages), (g / kStages) & 1);
+      };
+      auto pv_ready = [&](int g) {
+        return mbar_test(bar(kPFull + (g & 1)), (g >> 1) & 1) &&
+               mbar_test(bar(kVReady + g % kStages), (g / kStages) & 1);
       };
       while (ok && pi.next(pc)) {
         if (!wait_bar(bar(kQReady), piece & 1, ctl)) { ok = false; break; }
-        tc_fence_after();
-        const int n = pc.pe - pc.pa;
-        ok = issue_qk(it) && (n < 2 || issue_qk(it + 1));
-        for (int j = 0; j < n && ok; ++j) {
-          ok = issue_pv(it + j, j == 0) && (j + 2 >= n || issue_qk(it + j + 2));
+        const int n = pc.pe - pc.pa, end = it + n;
+        int gq = it, gp = it;
+        uint64_t idle_since = 0;
+        while (gp < end) {
+          bool prog = false;
+          if (gq < end && qk_ready(gq)) {
+            do_qk(gq++);
+            prog = true;
+          }
+          if (gp < gq && pv_ready(gp)) {
+            do_pv(gp, gp == it);
+            ++gp;
+            prog = true;
+          }
+          if (prog) {
+            idle_since = 0;
+            continue;
+          }
+          if (abort_s) { ok = false; break; }
+          const uint64_t t = now_ns();
+          if (idle_since == 0) {
+            idle_since = t;
+          } else if (t - idle_since > limit_ns) {
+            set_device_error(a.err, MLA_ERR_DEVICE_TIMEOUT);
+            abort_s = 1;
+            asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(ctl.peer_abort), "r"(1) : "memory");
+            ok = false;
+            break;
+          }
         }
         if (!ok) break;
         mma_commit(bar(kOFull));
@@ -342,60 +376,46 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         if (lane == 0) mbar_arrive(bar(kVReady + s));
       }
     }
-  } else if (warp == 3) {
-    // ------------------------------------------------------------ receive-buffer recycler
-    // After the PV of page g has consumed receive buffer g&1 (which held the peer's
-    // partial and then P), arm it for page g+2 and let the peer send into it.
-    if (lane == 0) {
-      PieceIter pi(sc, w);
-      Piece pc;
-      int g = 0;
-      bool ok = true;
-      const uint32_t peer_free = map_to_rank(bar(kPeerFree), peer);
-      while (ok && pi.next(pc)) {
-        for (int p = pc.pa; p < pc.pe; ++p, ++g) {
-          const int u = g & 1;
-          if (!wait_bar(bar(kPvDone + u), (g >> 1) & 1, ctl)) { ok = false; break; }
-          mbar_expect_tx(bar(kRxFull + u), kXBytes);
-          mbar_arrive_cluster(peer_free + u * 8);
-        }
-      }
-    }
-    __syncwarp();
-  } else {
-    // ------------------------------------------------------------ softmax warpgroup
-    const int row = tid - 128;             // head row = TMEM lane
+  } else if (warp >= 4) {
+    // ------------------------------------------------------------ softmax warpgroups
+    // Two warpgroups split every page's 64 score columns: warpgroup wg owns columns
+    // [32 wg, 32 wg + 32) of each head row (and the same half of its O columns); the
+    // two threads of a row exchange their half-row maxima through shared memory, so
+    // both apply the same running max.
+    const int sw = warp - 4;               // softmax warp 0..7
+    const int wg = sw >> 2;                // column half
     const int q = warp & 3;                // lane quadrant of this warp
+    const int row = 32 * q + lane;         // head row = TMEM lane
     const uint32_t lane_off = (uint32_t)(32 * q) << 16;
-    const uint32_t t_o = tmem + lane_off + kColO;
-    const uint32_t t_q = tmem + lane_off + kColQ;
+    const uint32_t t_o = tmem + lane_off + kColO + 128 * wg;  // this thread's half of the O row
+    const uint32_t t_q = tmem + lane_off + kColQ + 64 * wg;   // this thread's half of the q' latent columns
     const uint32_t rx_peer = map_to_rank(s_rx, peer);
     const uint32_t peer_rx_full = map_to_rank(bar(kRxFull), peer);
-    const bool sender = row == 0;
+    const bool sender = wg == 0 && row == 0;
     const float scale2 = a.scale * kLog2e;
-    uint8_t* txrow = smem + kSmemTx + row * 256;
+    uint8_t* txrow = smem + kSmemTx + row * kXRow;
+    const uint32_t peer_free = map_to_rank(bar(kPeerFree), peer);
+    const int sw2 = (row >> 1) & 3;  // chunk swizzle of 192-byte rows: XOR keeps groups of 4 chunks
+    float* hmax = reinterpret_cast<float*>(smem + kSmemHmax);  // [page parity][wg][row]
+    float* lsum = reinterpret_cast<float*>(smem + kSmemLsum);  // [wg][row]
     PieceIter pi(sc, w);
     Piece pc;
     int it = 0, piece = 0;
     bool ok = true;
-    float own0[64], own1[64];
+    float own0[32], own1[32];
 
-    // Stage A of global page g: load this CTA's partial scores, free the S buffer,
-    // scale to log2 units, and send them to the peer.
-    auto stage_a = [&](int g, float (&own)[64]) -> bool {
+    // Stage A of global page g: load this thread's half of the partial scores, free
+    // the S buffer, scale to log2 units, and send them to the peer.
+    auto stage_a = [&](int g, float (&own)[32]) -> bool {
       const int u = g & 1, k = g >> 1;
       if (!__all_sync(0xffffffffu, wait_bar(bar(kSFull + u), k & 1, ctl))) return false;
       tc_fence_after();
       {
-        uint32_t r0[32], r1[32];
-        tmem_ld32(tmem + lane_off + kColS + 64 * u, r0);
-        tmem_ld32(tmem + lane_off + kColS + 64 * u + 32, r1);
+        uint32_t r0[32];
+        tmem_ld32(tmem + lane_off + kColS + 64 * u + 32 * wg, r0);
         tmem_wait_ld();
 #pragma unroll
-        for (int c = 0; c < 32; ++c) {
-          own[c] = __uint_as_float(r0[c]) * scale2;
-          own[32 + c] = __uint_as_float(r1[c]) * scale2;
-        }
+        for (int c = 0; c < 32; ++c) own[c] = __uint_as_float(r0[c]) * scale2;
       }
       tc_fence_before();
       mbar_arrive(bar(kSFree + u));
@@ -405,16 +425,34 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         mbar_arrive(bar(kTxWritable));
       }
       if (!__all_sync(0xffffffffu, wait_bar(bar(kTxWritable), g & 1, ctl))) return false;
+      // 24-bit values (fp32 rounded to 15 mantissa bits), 4 per 12 bytes: this
+      // warpgroup's 32 values are 24 words = 6 chunks of 16 bytes.  Our own values
+      // are rounded the same way, so both CTAs add identical operands.
+      {
+        uint32_t wd[24];
 #pragma unroll
-      for (int c = 0; c < 16; ++c)
-        *reinterpret_cast<float4*>(txrow + ((c ^ (row & 7)) * 16)) =
-            make_float4(own[4 * c], own[4 * c + 1], own[4 * c + 2], own[4 * c + 3]);
+        for (int e = 0; e < 8; ++e) {
+          uint32_t t[4];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            t[i] = (__float_as_uint(own[4 * e + i]) + 0x80u) >> 8;
+            own[4 * e + i] = __uint_as_float(t[i] << 8);
+          }
+          wd[3 * e + 0] = t[0] | (t[1] << 24);
+          wd[3 * e + 1] = (t[1] >> 8) | (t[2] << 16);
+          wd[3 * e + 2] = (t[2] >> 16) | (t[3] << 8);
+        }
+#pragma unroll
+        for (int c = 0; c < 6; ++c)
+          *reinterpret_cast<uint4*>(txrow + (((6 * wg + c) ^ sw2) * 16)) =
+              make_uint4(wd[4 * c], wd[4 * c + 1], wd[4 * c + 2], wd[4 * c + 3]);
+      }
       fence_proxy_async();
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(kTxReady));
       bool good = true;
       if (sender) {
-        // Our rows are written, and the peer has freed and armed its receive buffer u.
+        // All rows are written, and the peer has freed and armed its receive buffer u.
         good = wait_bar(bar(kPeerFree + u), (k & 1) ^ 1, ctl) && wait_bar(bar(kTxReady), g & 1, ctl);
         if (good) bulk_copy_to_peer(rx_peer + u * kXBytes, s_tx, kXBytes, peer_rx_full + u * 8);
       }
@@ -424,16 +462,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     while (ok && pi.next(pc)) {
       const int b = pc.b, n = pc.pe - pc.pa;
       const int T = a.seqlens[b];
-      // ---- stage q' for this sequence: latent half -> TMEM, this CTA's 32 rope dims -> smem
+      // ---- stage q' for this sequence: latent half -> TMEM (split between the
+      // warpgroups), this CTA's 32 rope dims -> smem (64B swizzle)
       {
         uint32_t qv[16];
         const bool live = row < a.heads;
         const uint4* src = reinterpret_cast<const uint4*>(a.q + ((size_t)b * a.heads + (live ? row : 0)) * kDQK);
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {  // 8 x 32 dims of this CTA's 256 latent dims
+        for (int c = 0; c < 4; ++c) {  // 4 x 32 dims of this warpgroup's 128 latent dims
 #pragma unroll
           for (int k = 0; k < 4; ++k) {
-            const uint4 v = live ? src[(256 * rank) / 8 + c * 4 + k] : make_uint4(0, 0, 0, 0);
+            const uint4 v = live ? src[32 * rank + 16 * wg + 4 * c + k] : make_uint4(0, 0, 0, 0);
             qv[4 * k + 0] = v.x;
             qv[4 * k + 1] = v.y;
             qv[4 * k + 2] = v.z;
@@ -441,11 +480,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           }
           tmem_st16(t_q + c * 16, qv);
         }
-        uint8_t* qr = smem + kSmemQRope + row * 64;
+        if (wg == 0) {
+          uint8_t* qr = smem + kSmemQRope + row * 64;
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {  // 64B swizzle: 16-byte chunk c of row r at c ^ ((r >> 1) & 3)
-          const uint4 v = live ? src[kDLatent / 8 + 4 * rank + c] : make_uint4(0, 0, 0, 0);
-          *reinterpret_cast<uint4*>(qr + ((c ^ ((row >> 1) & 3)) * 16)) = v;
+          for (int c = 0; c < 4; ++c) {  // 64B swizzle: 16-byte chunk c of row r at c ^ ((r >> 1) & 3)
+            const uint4 v = live ? src[kDLatent / 8 + 4 * rank + c] : make_uint4(0, 0, 0, 0);
+            *reinterpret_cast<uint4*>(qr + ((c ^ ((row >> 1) & 3)) * 16)) = v;
+          }
         }
         tmem_wait_st();
         fence_proxy_async();
@@ -455,90 +496,113 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       float m = -INFINITY, l = 0.f;
       bool bad = false;
       int pid_next = page_of(a, b, pc.pa);
-      ok = (it & 1) ? stage_a(it, own1) : stage_a(it, own0);
       // Stage B of page j of this piece: add the peer's partial, online softmax, write P.
-      auto stage_b = [&](int j, float (&x)[64]) -> bool {
+      auto stage_b = [&](int j, float (&x)[32]) -> bool {
         const int g = it + j, u = g & 1, k = g >> 1, p = pc.pa + j;
-          if (!__all_sync(0xffffffffu, wait_bar(bar(kRxFull + u), k & 1, ctl))) return false;
-          {
-            const uint8_t* rxrow = smem + kSmemRx + u * kXBytes + row * 256;
+        if (!__all_sync(0xffffffffu, wait_bar(bar(kRxFull + u), k & 1, ctl))) return false;
+        {
+          const uint8_t* rxrow = smem + kSmemRx + u * kXBytes + row * kXRow;
+          uint32_t wd[24];
 #pragma unroll
-            for (int c = 0; c < 16; ++c) {
-              const float4 v = *reinterpret_cast<const float4*>(rxrow + ((c ^ (row & 7)) * 16));
-              // fp32 addition is commutative: both CTAs hold the same sums.
-              x[4 * c + 0] += v.x;
-              x[4 * c + 1] += v.y;
-              x[4 * c + 2] += v.z;
-              x[4 * c + 3] += v.w;
-            }
+          for (int c = 0; c < 6; ++c) {
+            const uint4 v = *reinterpret_cast<const uint4*>(rxrow + (((6 * wg + c) ^ sw2) * 16));
+            wd[4 * c] = v.x;
+            wd[4 * c + 1] = v.y;
+            wd[4 * c + 2] = v.z;
+            wd[4 * c + 3] = v.w;
           }
-          __syncwarp();
-          if (lane == 0) mbar_arrive(bar(kRxRead));
-          const int pid = pid_next;
-          if (j + 1 < n) pid_next = page_of(a, b, p + 1);  // used next page: latency off the chain
-          if ((unsigned)pid >= (unsigned)np) {
-            bad = true;
-            set_device_error(a.err, MLA_ERR_DEVICE_BAD_PAGE);
-          }
-          const int valid = min(kPage, T - p * kPage);
-          float tmax = -INFINITY;
 #pragma unroll
-          for (int c = 0; c < 64; ++c) {
-            x[c] = c < valid ? x[c] : -INFINITY;
-            tmax = fmaxf(tmax, x[c]);
+          for (int e = 0; e < 8; ++e) {
+            const uint32_t w0 = wd[3 * e], w1 = wd[3 * e + 1], w2 = wd[3 * e + 2];
+            // fp32 addition is commutative: both CTAs hold the same sums.
+            x[4 * e + 0] += __uint_as_float((w0 & 0xFFFFFFu) << 8);
+            x[4 * e + 1] += __uint_as_float(((w0 >> 24) | ((w1 & 0xFFFFu) << 8)) << 8);
+            x[4 * e + 2] += __uint_as_float(((w1 >> 16) | ((w2 & 0xFFu) << 16)) << 8);
+            x[4 * e + 3] += __uint_as_float((w2 >> 8) << 8);
           }
-          const float m_new = fmaxf(m, tmax);
-          const bool need = m_new > m + kRescaleThreshold;
-          const float alpha = need ? fast_exp2(m - m_new) : 1.f;
-          if (need) m = m_new;
-          if (__any_sync(0xffffffffu, need && j > 0)) {
-            // O must hold PV(g-1) before it is rescaled (rare path).
-            const int x = g - 1;
-            if (!__all_sync(0xffffffffu, wait_bar(bar(kODone + 2 * q + (x & 1)), (x >> 1) & 1, ctl))) return false;
-            tc_fence_after();
+        }
+        const int pid = pid_next;
+        if (j + 1 < n) pid_next = page_of(a, b, p + 1);  // used next page: latency off the chain
+        if ((unsigned)pid >= (unsigned)np) {
+          bad = true;
+          set_device_error(a.err, MLA_ERR_DEVICE_BAD_PAGE);
+        }
+        const int valid = min(kPage, T - p * kPage) - 32 * wg;  // valid columns of this half
+        float hm = -INFINITY;
+#pragma unroll
+        for (int c = 0; c < 32; ++c) {
+          x[c] = c < valid ? x[c] : -INFINITY;
+          hm = fmaxf(hm, x[c]);
+        }
+        hmax[((g & 1) * 2 + wg) * 128 + row] = hm;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(kXMax));
+        // Both halves published; this also certifies that every row of the receive
+        // buffer has been read: re-arm it for page g+2 and let the peer send into it.
+        if (!__all_sync(0xffffffffu, wait_bar(bar(kXMax), g & 1, ctl))) return false;
+        if (sender) {
+          mbar_expect_tx(bar(kRxFull + u), kXBytes);
+          mbar_arrive_cluster(peer_free + u * 8);
+        }
+        const float tmax = fmaxf(hm, hmax[((g & 1) * 2 + (wg ^ 1)) * 128 + row]);
+        const float m_new = fmaxf(m, tmax);
+        const bool need = m_new > m + kRescaleThreshold;
+        const float alpha = need ? fast_exp2(m - m_new) : 1.f;
+        if (need) m = m_new;
+        if (__any_sync(0xffffffffu, need && j > 0)) {
+          // O must hold PV(g-1) before it is rescaled (rare path).
+          const int x1 = g - 1;
+          if (!__all_sync(0xffffffffu, wait_bar(bar(kODone + 2 * sw + (x1 & 1)), (x1 >> 1) & 1, ctl))) return false;
+          tc_fence_after();
 #pragma unroll 1
-            for (int c = 0; c < 8; ++c) {
-              uint32_t r[32];
-              tmem_ld32(t_o + c * 32, r);
-              tmem_wait_ld();
-              uint32_t w0[16], w1[16];
+          for (int c = 0; c < 4; ++c) {
+            uint32_t r[32];
+            tmem_ld32(t_o + c * 32, r);
+            tmem_wait_ld();
+            uint32_t w0[16], w1[16];
 #pragma unroll
-              for (int e = 0; e < 16; ++e) {
-                w0[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
-                w1[e] = __float_as_uint(__uint_as_float(r[16 + e]) * alpha);
-              }
-              tmem_st16(t_o + c * 32, w0);
-              tmem_st16(t_o + c * 32 + 16, w1);
+            for (int e = 0; e < 16; ++e) {
+              w0[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
+              w1[e] = __float_as_uint(__uint_as_float(r[16 + e]) * alpha);
             }
-            tmem_wait_st();
-            tc_fence_before();
+            tmem_st16(t_o + c * 32, w0);
+            tmem_st16(t_o + c * 32 + 16, w1);
           }
-          l *= alpha;
-          uint32_t pk[32];
-          float rs = 0.f;
+          tmem_wait_st();
+          tc_fence_before();
+        }
+        l *= alpha;
+        uint32_t pk[16];
+        float rs = 0.f;
 #pragma unroll
-          for (int c = 0; c < 32; ++c) {
-            const float p0 = fast_exp2(x[2 * c] - m);
-            const float p1 = fast_exp2(x[2 * c + 1] - m);
-            rs += p0 + p1;
-            pk[c] = pack_bf16x2(p0, p1);
-          }
-          l += rs;
-          // Every row of the receive buffer has been read: overwrite it with P
-          // ([128 heads x 64 tokens] bf16, K-major, 128B swizzle: the PV A operand).
-          if (!__all_sync(0xffffffffu, wait_bar(bar(kRxRead), g & 1, ctl))) return false;
-          {
-            uint8_t* prow = smem + kSmemRx + u * kXBytes + row * 128;
+        for (int c = 0; c < 16; ++c) {
+          const float p0 = fast_exp2(x[2 * c] - m);
+          const float p1 = fast_exp2(x[2 * c + 1] - m);
+          rs += p0 + p1;
+          pk[c] = pack_bf16x2(p0, p1);
+        }
+        l += rs;
+        // P [128 heads x 64 tokens] bf16, K-major, 128B swizzle (the PV A operand):
+        // this thread's 4 chunks of its row.  Buffer u was last read by PV(g-2); the
+        // next completion on its barrier is PV(g), which needs this P, so the wait
+        // cannot fall two phases behind.
+        if (g >= 2) {
+          const int x2 = g - 2;
+          if (!__all_sync(0xffffffffu, wait_bar(bar(kODone + 2 * sw + (x2 & 1)), (x2 >> 1) & 1, ctl))) return false;
+        }
+        {
+          uint8_t* prow = smem + kSmemP + u * kPBytes + row * 128;
 #pragma unroll
-            for (int c = 0; c < 8; ++c)
-              *reinterpret_cast<uint4*>(prow + ((c ^ (row & 7)) * 16)) =
-                  make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
-          }
-          fence_proxy_async();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(bar(kPFull + u));
+          for (int c = 0; c < 4; ++c)
+            *reinterpret_cast<uint4*>(prow + (((4 * wg + c) ^ (row & 7)) * 16)) =
+                make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+        }
+        fence_proxy_async();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(kPFull + u));
         return true;
       };
+      ok = (it & 1) ? stage_a(it, own1) : stage_a(it, own0);
       for (int j = 0; j < n && ok; ++j) {
         const int g = it + j;
         if (j + 1 < n) {
@@ -548,11 +612,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         ok = (g & 1) ? stage_b(j, own1) : stage_b(j, own0);
       }
       if (!ok) break;
-      // ---- epilogue: O / l (this CTA's 256 dims), lse
+      // ---- epilogue: O / l (this thread's 128 of the CTA's 256 dims), lse
       if (!__all_sync(0xffffffffu, wait_bar(bar(kOFull), piece & 1, ctl))) { ok = false; break; }
       tc_fence_after();
-      const float inv = bad ? NAN : 1.f / l;
-      const float lse_v = bad ? NAN : (m + __log2f(l)) * kLn2;
+      lsum[wg * 128 + row] = l;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(kLSync));
+      if (!__all_sync(0xffffffffu, wait_bar(bar(kLSync), piece & 1, ctl))) { ok = false; break; }
+      const float l_row = lsum[row] + lsum[128 + row];
+      const float inv = bad ? NAN : 1.f / l_row;
+      const float lse_v = bad ? NAN : (m + __log2f(l_row)) * kLn2;
       const bool complete = pc.pa == 0 && pc.pe == sc.seq_start[b + 1] - sc.seq_start[b];
       float* obase;
       float* lbase;
@@ -565,19 +634,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         lbase = sc.part_lse + (size_t)slot * a.heads;
       }
 #pragma unroll 1
-      for (int c = 0; c < 8; ++c) {
+      for (int c = 0; c < 4; ++c) {
         uint32_t r[32];
         tmem_ld32(t_o + c * 32, r);
         tmem_wait_ld();
         if (row < a.heads) {
-          float4* dst = reinterpret_cast<float4*>(obase + (size_t)row * kDLatent + 256 * rank + 32 * c);
+          float4* dst = reinterpret_cast<float4*>(obase + (size_t)row * kDLatent + 256 * rank + 128 * wg + 32 * c);
 #pragma unroll
           for (int e = 0; e < 8; ++e)
             dst[e] = make_float4(__uint_as_float(r[4 * e]) * inv, __uint_as_float(r[4 * e + 1]) * inv,
                                  __uint_as_float(r[4 * e + 2]) * inv, __uint_as_float(r[4 * e + 3]) * inv);
         }
       }
-      if (rank == 0 && row < a.heads) lbase[row] = lse_v;
+      if (rank == 0 && wg == 0 && row < a.heads) lbase[row] = lse_v;
       tc_fence_before();
       it += n;
       ++piece;

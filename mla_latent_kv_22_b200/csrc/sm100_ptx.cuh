@@ -39,6 +39,17 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
+// Non-blocking test of a phase.
+__device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.test_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n"
+      " selp.b32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
 // Bounded wait: spins at most `limit` times, then records MLA_ERR_DEVICE_TIMEOUT
 // in *err (and in *abort, shared by the CTA) and returns false.  Never traps.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, int limit, int* err, volatile int* abort) {
