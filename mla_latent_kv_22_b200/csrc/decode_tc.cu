@@ -10,9 +10,12 @@
 // (latent [256r, 256r+256) plus rope [512+32r, 512+32r+32)).  Each CTA therefore
 // loads only its part of every row (HBM and L2 traffic 1x), computes a partial S,
 // and the two partials are exchanged through distributed shared memory by bulk
-// copies and added, so both CTAs run a bit-identical softmax.  Each exchanged score
-// is the fp32 value rounded to 24 bits (sign, exponent, 15 mantissa bits; relative
-// error <= 2^-16), 4 values in 12 bytes: 24 KB per page each way.
+// copies and added.  Each exchanged score is the top 3 bytes of its fp32 pattern
+// (sign, exponent, 15 mantissa bits), the dropped byte refilled with its mid-point
+// (relative error <= 2^-16), 4 values in 12 bytes: 24 KB per page each way.  Each
+// CTA adds its own exact partial to the peer's, so the two softmaxes agree to that
+// rounding; each CTA normalises its half of O by its own row sums, and rank 0
+// writes the lse.
 //
 // Pipeline.  The exchange has a long latency, so the softmax threads are software
 // pipelined: in each iteration they first send page j+1's partial (stage A) and
@@ -21,9 +24,11 @@
 // written (bf16) to shared memory and read from there by the PV MMA, which frees
 // each S buffer as soon as it has been loaded, so score MMAs run ahead.
 //
-// Roles (384 threads): warp 0 issues TMA loads, warp 1 allocates TMEM and issues
-// MMAs (whichever of the next score MMA and the next PV is ready first), warp 2
-// zeroes value rows past the sequence end before PV reads them, warp 3 idles,
+// Roles (384 threads): warp 0 issues TMA loads (and L2 prefetches a few pages
+// ahead), warp 1 allocates TMEM and issues MMAs (whichever of the next score MMA
+// and the next PV is ready first), warp 2 zeroes value rows past the sequence end
+// before PV reads them and hands read receive buffers back to the peer, warp 3
+// copies each page's packed partial scores to the peer, and
 // warps 4..11 are two softmax warpgroups (one thread per
 // head row = TMEM lane, each warpgroup half of every page's columns) that stage q',
 // exchange partial scores, run the online softmax (log2 domain, lazy rescale by at
@@ -31,10 +36,10 @@
 //
 // TMEM (512 columns): O [0,256) fp32, S double buffer [256,320) [320,384) fp32,
 // q' latent half [384,512) as bf16 pairs (the A operand of the latent QK^T).
-// Shared memory: 3 stages x (4 latent boxes [64 tokens x 64 dims], 128B swizzle:
+// Shared memory: 4 stages x (4 latent boxes [64 tokens x 64 dims], 128B swizzle:
 // K-major B of QK^T and MN-major B of PV; 1 rope box [64 tokens x 32 dims], 64B
-// swizzle); this CTA's rope part of q' [128 x 32] (64B swizzle, A operand); one
-// 24 KB send buffer; two 24 KB receive buffers; two 16 KB P buffers (128B swizzle).
+// swizzle); this CTA's rope part of q' [128 x 32] (64B swizzle, A operand); a 24 KB
+// send and a 24 KB receive buffer; a 16 KB P buffer (128B swizzle).
 //
 // Every mbarrier wait is bounded by a time limit; on expiry the kernel records
 // MLA_ERR_DEVICE_TIMEOUT, tells the peer CTA to stop, drains its own TMA, bulk-copy
@@ -54,20 +59,20 @@ namespace {
 using namespace sm100;
 
 constexpr int kThreads = 384;
-constexpr int kStages = 3;
+constexpr int kStages = 4;
 constexpr int kLatBox = 64 * 128;                 // [64 rows x 64 bf16], 128B swizzle
 constexpr int kRopeBox = 64 * 64;                 // [64 rows x 32 bf16], 64B swizzle
 constexpr int kStageBytes = 4 * kLatBox + kRopeBox;  // 36864
 constexpr int kXRow = 64 * 3;                     // one head row of partial scores, 24 bits per value
 constexpr int kXBytes = 128 * kXRow;              // 24576: [128 heads x 64 tokens] partial scores
 constexpr int kPBytes = 128 * 128;                // [128 heads x 64 tokens] bf16 P
-constexpr int kSmemQRope = kStages * kStageBytes;             // 110592
-constexpr int kSmemTx = kSmemQRope + 128 * 64;                // 118784
-constexpr int kSmemRx = kSmemTx + kXBytes;                    // 143360: 2 receive buffers
-constexpr int kSmemP = kSmemRx + 2 * kXBytes;                 // 192512: 2 P buffers (1024-aligned)
-constexpr int kSmemHmax = kSmemP + 2 * kPBytes;               // 225280: half-row maxima [2][2][128]
-constexpr int kSmemLsum = kSmemHmax + 2 * 2 * 128 * 4;        // 227328: half-row sums [2][128]
-constexpr int kSmemBytes = kSmemLsum + 2 * 128 * 4;           // 228352
+constexpr int kSmemQRope = kStages * kStageBytes;             // 147456
+constexpr int kSmemTx = kSmemQRope + 128 * 64;                // 155648
+constexpr int kSmemRx = kSmemTx + kXBytes;                    // 180224: receive buffer
+constexpr int kSmemP = kSmemRx + kXBytes;                     // 204800: P (1024-aligned)
+constexpr int kSmemHmax = kSmemP + kPBytes;                   // 221184: half-row maxima [2][2][128]
+constexpr int kSmemLsum = kSmemHmax + 2 * 2 * 128 * 4;        // 223232: half-row sums [2][128]
+constexpr int kSmemBytes = kSmemLsum + 2 * 128 * 4;           // 224256
 constexpr int kSmemAlloc = kSmemBytes + 1024;                 // + alignment slack
 
 constexpr uint32_t kTmemCols = 512;
@@ -77,6 +82,7 @@ constexpr uint32_t kIdescQK = idesc_bf16_f32(128, 64, 0, 0);   // A K-major (TME
 constexpr uint32_t kIdescPV = idesc_bf16_f32(128, 256, 0, 1);  // A (P, smem) K-major, B MN-major
 
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: P may reach 2^8 before O is rescaled
+constexpr int kPrefetch = 4;               // pages pulled into L2 ahead of the stage loads
 
 enum Bar {
   kKvFull = 0,
@@ -85,14 +91,14 @@ enum Bar {
   kSFull = kVReady + kStages,
   kSFree = kSFull + 2,
   kPFull = kSFree + 2,
-  kRxFull = kPFull + 2,
-  kPeerFree = kRxFull + 2,
-  kTxWritable = kPeerFree + 2,
+  kRxFull = kPFull + 1,
+  kPeerFree = kRxFull + 1,
+  kTxWritable = kPeerFree + 1,
   kTxReady = kTxWritable + 1,
-  kXMax = kTxReady + 1,   // half-row maxima published (and the receive buffer fully read)
-  kLSync = kXMax + 1,     // half-row sums published (epilogue)
-  kODone = kLSync + 1,    // [softmax warp][PV parity]: 16 barriers
-  kOFull = kODone + 16,
+  kXMax = kTxReady + 1,   // [page parity] half-row maxima published, receive buffer read
+  kLSync = kXMax + 2,     // half-row sums published (epilogue)
+  kODone = kLSync + 1,    // PV(g) complete: O holds page g, P may be rewritten
+  kOFull = kODone + 1,
   kQReady = kOFull + 1,
   kDrain = kQReady + 1,
   kNumBars = kDrain + 1
@@ -137,9 +143,9 @@ struct Ctl {
   uint64_t limit_ns;
 };
 
-// Bounded wait on a local mbarrier phase; on timeout or abort returns false.
-__device__ __noinline__ bool wait_bar(uint32_t bar, uint32_t parity, const Ctl& c) {
-  if (mbar_try_wait(bar, parity)) return true;
+// Bounded wait on a local mbarrier phase; on timeout or abort returns false.  The
+// first probe is inline; only a wait that does not complete at once makes a call.
+__device__ __noinline__ bool wait_bar_slow(uint32_t bar, uint32_t parity, const Ctl& c) {
   const uint64_t t0 = now_ns();
   for (uint32_t i = 1;; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
@@ -153,6 +159,9 @@ __device__ __noinline__ bool wait_bar(uint32_t bar, uint32_t parity, const Ctl& 
       }
     }
   }
+}
+__device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, const Ctl& c) {
+  return mbar_try_wait(bar, parity) || wait_bar_slow(bar, parity, c);
 }
 
 // Spin (bounded by time, ignoring the abort flag) until a phase completes: used only
@@ -198,21 +207,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     for (int u = 0; u < 2; ++u) {
       mbar_init(bar(kSFull + u), 1);      // MMA commit
       mbar_init(bar(kSFree + u), 256);    // every softmax thread has loaded its half of S
-      mbar_init(bar(kPFull + u), 8);      // one arrival per softmax warp
-      mbar_init(bar(kRxFull + u), 1);     // armed (expect_tx) here, bytes from the peer
-      mbar_init(bar(kPeerFree + u), 1);   // the peer's receive buffer u is read and re-armed
     }
+    mbar_init(bar(kPFull), 8);      // one arrival per softmax warp
+    mbar_init(bar(kRxFull), 1);     // armed (expect_tx) here, bytes from the peer
+    mbar_init(bar(kPeerFree), 1);   // the peer's receive buffer is read and re-armed
     mbar_init(bar(kTxWritable), 1);
     mbar_init(bar(kTxReady), 8);
-    mbar_init(bar(kXMax), 8);
+    for (int u = 0; u < 2; ++u) mbar_init(bar(kXMax + u), 8);
     mbar_init(bar(kLSync), 8);
-    for (int q = 0; q < 16; ++q) mbar_init(bar(kODone + q), 1);
+    mbar_init(bar(kODone), 1);
     mbar_init(bar(kOFull), 1);
     mbar_init(bar(kQReady), 256);
     mbar_init(bar(kDrain), 1);
-    // The first round of both receive buffers is armed before the peer may send.
-    mbar_expect_tx(bar(kRxFull + 0), kXBytes);
-    mbar_expect_tx(bar(kRxFull + 1), kXBytes);
+    // The receive buffer is armed for page 0 before the peer may send.
+    mbar_expect_tx(bar(kRxFull), kXBytes);
     fence_mbar_init();
     tma_prefetch_desc(&kv_map);
     tma_prefetch_desc(&rope_map);
@@ -235,11 +243,34 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       Piece pc;
       int it = 0;
       bool ok = true;
+      // A second walk over the same pages runs kPrefetch pages ahead and pulls this
+      // CTA's part of each page into L2, so the loads into the stage ring (whose
+      // depth is bounded by shared memory) see L2 rather than HBM latency.
+      PieceIter pf(sc, w);
+      Piece fc;
+      bool fvalid = pf.next(fc);
+      int fp = fvalid ? fc.pa : 0;
+      auto prefetch_next = [&]() {
+        if (!fvalid) return;
+        const int pid = page_of(a, fc.b, fp);
+        if ((unsigned)pid < (unsigned)np) {
+          const int y = pid * kPage;
+#pragma unroll
+          for (int i = 0; i < 4; ++i) tma_prefetch_l2_2d(&kv_map, 256 * rank + 64 * i, y);
+          tma_prefetch_l2_2d(&rope_map, kDLatent + 32 * rank, y);
+        }
+        if (++fp >= fc.pe) {
+          fvalid = pf.next(fc);
+          fp = fvalid ? fc.pa : 0;
+        }
+      };
+      for (int i = 0; i < kPrefetch; ++i) prefetch_next();
       while (ok && pi.next(pc)) {
         for (int p = pc.pa; p < pc.pe; ++p, ++it) {
           const int s = it % kStages;
+          int pid = page_of(a, pc.b, p);  // table read issued before the wait, off the critical path
+          prefetch_next();
           if (!wait_bar(bar(kKvEmpty + s), ((it / kStages) & 1) ^ 1, ctl)) { ok = false; break; }
-          int pid = page_of(a, pc.b, p);
           if ((unsigned)pid >= (unsigned)np) pid = 0;  // reported by the softmax warps; load something valid
           if (a.withhold_arrive && w == 0 && rank == 0 && it == 1) continue;  // timeout test: never arrives
           const uint32_t dst = sbase + s * kStageBytes;
@@ -265,9 +296,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       Piece pc;
       int it = 0, piece = 0;
       bool ok = true;
-      // Issues whichever is ready first: the next score MMA (its S buffer freed and its
-      // page loaded) or the next PV (its P written and its value rows cleaned), so score
-      // MMAs never queue behind a PV that waits for the softmax.
       auto do_qk = [&](int g) {
         const int s = g % kStages, u = g & 1;
         tc_fence_after();
@@ -284,26 +312,29 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         mma_commit(bar(kSFull + u));
       };
       auto do_pv = [&](int g, bool first) {
-        const int s = g % kStages, u = g & 1;
+        const int s = g % kStages;
         tc_fence_after();
         const uint32_t vbase = sbase + s * kStageBytes;
-        const uint32_t pbase = s_p + u * kPBytes;
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
-          mma_ss(tmem + kColO, desc_sw128(pbase + kk * 32, 16, 1024), desc_sw128(vbase + kk * 2048, 8192, 1024),
+          mma_ss(tmem + kColO, desc_sw128(s_p + kk * 32, 16, 1024), desc_sw128(vbase + kk * 2048, 8192, 1024),
                  kIdescPV, (first && kk == 0) ? 0u : 1u);
         mma_commit(bar(kKvEmpty + s));
-        // PV(g) is tracked on the barriers of its parity: the next completion there
-        // is PV(g+2), which needs P(g+2), so a waiter is never two phases behind.
-#pragma unroll
-        for (int q = 0; q < 8; ++q) mma_commit(bar(kODone + 2 * q + u));
+        // The next completion of ODone after PV(g) is PV(g+1), which needs P(g+1),
+        // which is written only after every softmax warp has seen PV(g) done.
+        mma_commit(bar(kODone));
       };
+      // Issues whichever is ready first: the next score MMA (its S buffer freed and its
+      // page loaded) or the next PV (its P written and its value rows cleaned), so score
+      // MMAs run up to two pages ahead and never queue behind a PV that waits for the
+      // softmax.  When neither is ready the thread sleeps on the next P (a bounded,
+      // hinted try_wait), leaving the issue slots to the softmax warps.
       auto qk_ready = [&](int g) {
         return (g < 2 || mbar_test(bar(kSFree + (g & 1)), ((g - 2) >> 1) & 1)) &&
                mbar_test(bar(kKvFull + g % kStages), (g / kStages) & 1);
       };
       auto pv_ready = [&](int g) {
-        return mbar_test(bar(kPFull + (g & 1)), (g >> 1) & 1) &&
+        return mbar_test(bar(kPFull), g & 1) &&
                mbar_test(bar(kVReady + g % kStages), (g / kStages) & 1);
       };
       while (ok && pi.next(pc)) {
@@ -311,21 +342,27 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         const int n = pc.pe - pc.pa, end = it + n;
         int gq = it, gp = it;
         uint64_t idle_since = 0;
+        uint32_t idle = 0;
         while (gp < end) {
+          // PV first: it frees a stage (stage residency bounds the page rate) and the
+          // tensor pipe runs MMAs in issue order.
           bool prog = false;
-          if (gq < end && qk_ready(gq)) {
-            do_qk(gq++);
-            prog = true;
-          }
           if (gp < gq && pv_ready(gp)) {
             do_pv(gp, gp == it);
             ++gp;
             prog = true;
           }
+          if (gq < end && qk_ready(gq)) {
+            do_qk(gq++);
+            prog = true;
+          }
           if (prog) {
             idle_since = 0;
+            idle = 0;
             continue;
           }
+          if (gp < gq) mbar_try_wait_hint(bar(kPFull), gp & 1, 100);
+          if ((++idle & 15) != 0) continue;
           if (abort_s) { ok = false; break; }
           const uint64_t t = now_ns();
           if (idle_since == 0) {
@@ -349,7 +386,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     }
     __syncwarp();
   } else if (warp == 2) {
-    // ------------------------------------------------------------ tail rows of V
+    // ------------------------------------------------------------ tail rows of V,
+    // and receive buffers handed back to the peer
+    const uint32_t peer_free = map_to_rank(bar(kPeerFree), peer);
     PieceIter pi(sc, w);
     Piece pc;
     int it = 0;
@@ -374,8 +413,44 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(bar(kVReady + s));
+        // Every softmax warp has read the receive buffer (it published its half-row
+        // maxima after the read): re-arm it for page it+1 and let the peer send.  XMax
+        // is per page parity, so its next completion on this parity needs page it+2,
+        // which the peer can only send after this: the wait cannot fall behind.
+        if (!__all_sync(0xffffffffu, wait_bar(bar(kXMax + (it & 1)), (it >> 1) & 1, ctl))) { ok = false; break; }
+        if (lane == 0) {
+          mbar_expect_tx(bar(kRxFull), kXBytes);
+          mbar_arrive_cluster(peer_free);
+        }
       }
     }
+  } else if (warp == 3) {
+    // ------------------------------------------------------------ score sender:
+    // copies each page's packed partial scores into the peer's receive buffer
+    if (lane == 0) {
+      const uint32_t rx_peer = map_to_rank(s_rx, peer);
+      const uint32_t peer_rx_full = map_to_rank(bar(kRxFull), peer);
+      mbar_arrive(bar(kTxWritable));  // the send buffer starts free
+      PieceIter pi(sc, w);
+      Piece pc;
+      int it = 0;
+      bool ok = true;
+      while (ok && pi.next(pc)) {
+        for (int p = pc.pa; p < pc.pe; ++p, ++it) {
+          // All 8 softmax warps wrote their rows, and the peer has read page it-1 out of
+          // its receive buffer and re-armed it (the buffer starts armed for page 0).
+          if (!wait_bar(bar(kTxReady), it & 1, ctl) || (it > 0 && !wait_bar(bar(kPeerFree), (it - 1) & 1, ctl))) {
+            ok = false;
+            break;
+          }
+          bulk_copy_to_peer(rx_peer, s_tx, kXBytes, peer_rx_full);
+          bulk_wait_read_all();           // the copy has read the send buffer
+          mbar_arrive(bar(kTxWritable));  // the softmax may write the next page into it
+        }
+      }
+      bulk_wait_all();  // our copies into the peer have landed
+    }
+    __syncwarp();
   } else if (warp >= 4) {
     // ------------------------------------------------------------ softmax warpgroups
     // Two warpgroups split every page's 64 score columns: warpgroup wg owns columns
@@ -389,12 +464,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     const uint32_t lane_off = (uint32_t)(32 * q) << 16;
     const uint32_t t_o = tmem + lane_off + kColO + 128 * wg;  // this thread's half of the O row
     const uint32_t t_q = tmem + lane_off + kColQ + 64 * wg;   // this thread's half of the q' latent columns
-    const uint32_t rx_peer = map_to_rank(s_rx, peer);
-    const uint32_t peer_rx_full = map_to_rank(bar(kRxFull), peer);
-    const bool sender = wg == 0 && row == 0;
-    const float scale2 = a.scale * kLog2e;
+    // Scores stay unscaled (raw q'.k) until the exponent: a negative scale is moved
+    // into q' as an exact sign flip, so max over raw scores is max over scaled ones
+    // and each P costs one FFMA and one EX2.
+    const float scale2 = fabsf(a.scale) * kLog2e;
+    const uint32_t qsign = a.scale < 0.f ? 0x80008000u : 0u;
+    const float thr_raw = scale2 > 0.f ? kRescaleThreshold / scale2 : INFINITY;
     uint8_t* txrow = smem + kSmemTx + row * kXRow;
-    const uint32_t peer_free = map_to_rank(bar(kPeerFree), peer);
     const int sw2 = (row >> 1) & 3;  // chunk swizzle of 192-byte rows: XOR keeps groups of 4 chunks
     float* hmax = reinterpret_cast<float*>(smem + kSmemHmax);  // [page parity][wg][row]
     float* lsum = reinterpret_cast<float*>(smem + kSmemLsum);  // [wg][row]
@@ -405,42 +481,29 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     float own0[32], own1[32];
 
     // Stage A of global page g: load this thread's half of the partial scores, free
-    // the S buffer, scale to log2 units, and send them to the peer.
+    // the S buffer, and send them to the peer.
     auto stage_a = [&](int g, float (&own)[32]) -> bool {
       const int u = g & 1, k = g >> 1;
       if (!__all_sync(0xffffffffu, wait_bar(bar(kSFull + u), k & 1, ctl))) return false;
       tc_fence_after();
-      {
-        uint32_t r0[32];
-        tmem_ld32(tmem + lane_off + kColS + 64 * u + 32 * wg, r0);
-        tmem_wait_ld();
-#pragma unroll
-        for (int c = 0; c < 32; ++c) own[c] = __uint_as_float(r0[c]) * scale2;
-      }
+      uint32_t r0[32];
+      tmem_ld32(tmem + lane_off + kColS + 64 * u + 32 * wg, r0);
+      tmem_wait_ld();
       tc_fence_before();
       mbar_arrive(bar(kSFree + u));
-      // The previous page's copy out of the send buffer must have finished reading it.
-      if (sender) {
-        bulk_wait_read_all();
-        mbar_arrive(bar(kTxWritable));
-      }
+#pragma unroll
+      for (int c = 0; c < 32; ++c) own[c] = __uint_as_float(r0[c]);
+      // The previous page's copy out of the send buffer has finished reading it.
       if (!__all_sync(0xffffffffu, wait_bar(bar(kTxWritable), g & 1, ctl))) return false;
-      // 24-bit values (fp32 rounded to 15 mantissa bits), 4 per 12 bytes: this
-      // warpgroup's 32 values are 24 words = 6 chunks of 16 bytes.  Our own values
-      // are rounded the same way, so both CTAs add identical operands.
+      // Each value is sent as the top 3 bytes of its fp32 pattern; 4 values a, b, c, d
+      // travel as [a1 a2 a3 d1] [b1 b2 b3 d2] [c1 c2 c3 d3], 32 values = 6 chunks.
       {
         uint32_t wd[24];
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
-          uint32_t t[4];
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            t[i] = (__float_as_uint(own[4 * e + i]) + 0x80u) >> 8;
-            own[4 * e + i] = __uint_as_float(t[i] << 8);
-          }
-          wd[3 * e + 0] = t[0] | (t[1] << 24);
-          wd[3 * e + 1] = (t[1] >> 8) | (t[2] << 16);
-          wd[3 * e + 2] = (t[2] >> 16) | (t[3] << 8);
+          wd[3 * e + 0] = __byte_perm(r0[4 * e + 0], r0[4 * e + 3], 0x5321);
+          wd[3 * e + 1] = __byte_perm(r0[4 * e + 1], r0[4 * e + 3], 0x6321);
+          wd[3 * e + 2] = __byte_perm(r0[4 * e + 2], r0[4 * e + 3], 0x7321);
         }
 #pragma unroll
         for (int c = 0; c < 6; ++c)
@@ -450,13 +513,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       fence_proxy_async();
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(kTxReady));
-      bool good = true;
-      if (sender) {
-        // All rows are written, and the peer has freed and armed its receive buffer u.
-        good = wait_bar(bar(kPeerFree + u), (k & 1) ^ 1, ctl) && wait_bar(bar(kTxReady), g & 1, ctl);
-        if (good) bulk_copy_to_peer(rx_peer + u * kXBytes, s_tx, kXBytes, peer_rx_full + u * 8);
-      }
-      return __all_sync(0xffffffffu, good);
+      return true;
     };
 
     while (ok && pi.next(pc)) {
@@ -473,10 +530,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int k = 0; k < 4; ++k) {
             const uint4 v = live ? src[32 * rank + 16 * wg + 4 * c + k] : make_uint4(0, 0, 0, 0);
-            qv[4 * k + 0] = v.x;
-            qv[4 * k + 1] = v.y;
-            qv[4 * k + 2] = v.z;
-            qv[4 * k + 3] = v.w;
+            qv[4 * k + 0] = v.x ^ qsign;
+            qv[4 * k + 1] = v.y ^ qsign;
+            qv[4 * k + 2] = v.z ^ qsign;
+            qv[4 * k + 3] = v.w ^ qsign;
           }
           tmem_st16(t_q + c * 16, qv);
         }
@@ -484,7 +541,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           uint8_t* qr = smem + kSmemQRope + row * 64;
 #pragma unroll
           for (int c = 0; c < 4; ++c) {  // 64B swizzle: 16-byte chunk c of row r at c ^ ((r >> 1) & 3)
-            const uint4 v = live ? src[kDLatent / 8 + 4 * rank + c] : make_uint4(0, 0, 0, 0);
+            uint4 v = live ? src[kDLatent / 8 + 4 * rank + c] : make_uint4(0, 0, 0, 0);
+            v.x ^= qsign;
+            v.y ^= qsign;
+            v.z ^= qsign;
+            v.w ^= qsign;
             *reinterpret_cast<uint4*>(qr + ((c ^ ((row >> 1) & 3)) * 16)) = v;
           }
         }
@@ -493,15 +554,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         tc_fence_before();
         mbar_arrive(bar(kQReady));
       }
-      float m = -INFINITY, l = 0.f;
+      float m = -INFINITY, l = 0.f;  // running max of raw scores, running sum
       bool bad = false;
       int pid_next = page_of(a, b, pc.pa);
       // Stage B of page j of this piece: add the peer's partial, online softmax, write P.
       auto stage_b = [&](int j, float (&x)[32]) -> bool {
         const int g = it + j, u = g & 1, k = g >> 1, p = pc.pa + j;
-        if (!__all_sync(0xffffffffu, wait_bar(bar(kRxFull + u), k & 1, ctl))) return false;
+        if (!__all_sync(0xffffffffu, wait_bar(bar(kRxFull), g & 1, ctl))) return false;
         {
-          const uint8_t* rxrow = smem + kSmemRx + u * kXBytes + row * kXRow;
+          const uint8_t* rxrow = smem + kSmemRx + row * kXRow;
           uint32_t wd[24];
 #pragma unroll
           for (int c = 0; c < 6; ++c) {
@@ -511,14 +572,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             wd[4 * c + 2] = v.z;
             wd[4 * c + 3] = v.w;
           }
+          // The dropped low byte is refilled with 0x80 (mid-point): relative error <= 2^-16.
+          constexpr uint32_t kMid = 0x80808080u;
 #pragma unroll
           for (int e = 0; e < 8; ++e) {
             const uint32_t w0 = wd[3 * e], w1 = wd[3 * e + 1], w2 = wd[3 * e + 2];
-            // fp32 addition is commutative: both CTAs hold the same sums.
-            x[4 * e + 0] += __uint_as_float((w0 & 0xFFFFFFu) << 8);
-            x[4 * e + 1] += __uint_as_float(((w0 >> 24) | ((w1 & 0xFFFFu) << 8)) << 8);
-            x[4 * e + 2] += __uint_as_float(((w1 >> 16) | ((w2 & 0xFFu) << 16)) << 8);
-            x[4 * e + 3] += __uint_as_float((w2 >> 8) << 8);
+            x[4 * e + 0] += __uint_as_float(__byte_perm(w0, kMid, 0x2104));
+            x[4 * e + 1] += __uint_as_float(__byte_perm(w1, kMid, 0x2104));
+            x[4 * e + 2] += __uint_as_float(__byte_perm(w2, kMid, 0x2104));
+            const uint32_t t0 = __byte_perm(w0, kMid, 0x0034);  // [0x80, d1, -, -]
+            const uint32_t t1 = __byte_perm(w1, w2, 0x0073);    // [d2, d3, -, -]
+            x[4 * e + 3] += __uint_as_float(__byte_perm(t0, t1, 0x5410));
           }
         }
         const int pid = pid_next;
@@ -528,31 +592,26 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           set_device_error(a.err, MLA_ERR_DEVICE_BAD_PAGE);
         }
         const int valid = min(kPage, T - p * kPage) - 32 * wg;  // valid columns of this half
-        float hm = -INFINITY;
+        const bool ragged = valid < 32;                          // only a sequence's last page
+        if (ragged) {
 #pragma unroll
-        for (int c = 0; c < 32; ++c) {
-          x[c] = c < valid ? x[c] : -INFINITY;
-          hm = fmaxf(hm, x[c]);
+          for (int c = 0; c < 32; ++c) x[c] = c < valid ? x[c] : -INFINITY;
         }
-        hmax[((g & 1) * 2 + wg) * 128 + row] = hm;
+        float hm = x[0];
+#pragma unroll
+        for (int c = 1; c < 32; ++c) hm = fmaxf(hm, x[c]);
+        hmax[(u * 2 + wg) * 128 + row] = hm;
         __syncwarp();
-        if (lane == 0) mbar_arrive(bar(kXMax));
-        // Both halves published; this also certifies that every row of the receive
-        // buffer has been read: re-arm it for page g+2 and let the peer send into it.
-        if (!__all_sync(0xffffffffu, wait_bar(bar(kXMax), g & 1, ctl))) return false;
-        if (sender) {
-          mbar_expect_tx(bar(kRxFull + u), kXBytes);
-          mbar_arrive_cluster(peer_free + u * 8);
-        }
-        const float tmax = fmaxf(hm, hmax[((g & 1) * 2 + (wg ^ 1)) * 128 + row]);
+        if (lane == 0) mbar_arrive(bar(kXMax + u));
+        if (!__all_sync(0xffffffffu, wait_bar(bar(kXMax + u), k & 1, ctl))) return false;
+        const float tmax = fmaxf(hm, hmax[(u * 2 + (wg ^ 1)) * 128 + row]);
         const float m_new = fmaxf(m, tmax);
-        const bool need = m_new > m + kRescaleThreshold;
-        const float alpha = need ? fast_exp2(m - m_new) : 1.f;
+        const bool need = !(m_new <= m + thr_raw);  // also true while m is -inf
+        const float alpha = !need ? 1.f : (m == -INFINITY ? 0.f : fast_exp2((m - m_new) * scale2));
         if (need) m = m_new;
         if (__any_sync(0xffffffffu, need && j > 0)) {
           // O must hold PV(g-1) before it is rescaled (rare path).
-          const int x1 = g - 1;
-          if (!__all_sync(0xffffffffu, wait_bar(bar(kODone + 2 * sw + (x1 & 1)), (x1 >> 1) & 1, ctl))) return false;
+          if (!__all_sync(0xffffffffu, wait_bar(bar(kODone), (g - 1) & 1, ctl))) return false;
           tc_fence_after();
 #pragma unroll 1
           for (int c = 0; c < 4; ++c) {
@@ -572,26 +631,30 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           tc_fence_before();
         }
         l *= alpha;
-        uint32_t pk[16];
-        float rs = 0.f;
+        const float ms = m * scale2;
 #pragma unroll
-        for (int c = 0; c < 16; ++c) {
-          const float p0 = fast_exp2(x[2 * c] - m);
-          const float p1 = fast_exp2(x[2 * c + 1] - m);
-          rs += p0 + p1;
-          pk[c] = pack_bf16x2(p0, p1);
+        for (int c = 0; c < 32; ++c) x[c] = fast_exp2(fmaf(x[c], scale2, -ms));
+        if (ragged) {  // a zero scale turns -inf into NaN above
+#pragma unroll
+          for (int c = 0; c < 32; ++c) x[c] = c < valid ? x[c] : 0.f;
         }
-        l += rs;
+        float rs0 = 0.f, rs1 = 0.f, rs2 = 0.f, rs3 = 0.f;
+#pragma unroll
+        for (int c = 0; c < 32; c += 4) {
+          rs0 += x[c];
+          rs1 += x[c + 1];
+          rs2 += x[c + 2];
+          rs3 += x[c + 3];
+        }
+        l += (rs0 + rs1) + (rs2 + rs3);
+        uint32_t pk[16];
+#pragma unroll
+        for (int c = 0; c < 16; ++c) pk[c] = pack_bf16x2(x[2 * c], x[2 * c + 1]);
         // P [128 heads x 64 tokens] bf16, K-major, 128B swizzle (the PV A operand):
-        // this thread's 4 chunks of its row.  Buffer u was last read by PV(g-2); the
-        // next completion on its barrier is PV(g), which needs this P, so the wait
-        // cannot fall two phases behind.
-        if (g >= 2) {
-          const int x2 = g - 2;
-          if (!__all_sync(0xffffffffu, wait_bar(bar(kODone + 2 * sw + (x2 & 1)), (x2 >> 1) & 1, ctl))) return false;
-        }
+        // this thread's 4 chunks of its row.  The buffer was last read by PV(g-1).
+        if (g >= 1 && !__all_sync(0xffffffffu, wait_bar(bar(kODone), (g - 1) & 1, ctl))) return false;
         {
-          uint8_t* prow = smem + kSmemP + u * kPBytes + row * 128;
+          uint8_t* prow = smem + kSmemP + row * 128;
 #pragma unroll
           for (int c = 0; c < 4; ++c)
             *reinterpret_cast<uint4*>(prow + (((4 * wg + c) ^ (row & 7)) * 16)) =
@@ -599,7 +662,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         }
         fence_proxy_async();
         __syncwarp();
-        if (lane == 0) mbar_arrive(bar(kPFull + u));
+        if (lane == 0) mbar_arrive(bar(kPFull));
         return true;
       };
       ok = (it & 1) ? stage_a(it, own1) : stage_a(it, own0);
@@ -621,7 +684,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       if (!__all_sync(0xffffffffu, wait_bar(bar(kLSync), piece & 1, ctl))) { ok = false; break; }
       const float l_row = lsum[row] + lsum[128 + row];
       const float inv = bad ? NAN : 1.f / l_row;
-      const float lse_v = bad ? NAN : (m + __log2f(l_row)) * kLn2;
+      const float lse_v = bad ? NAN : (m * scale2 + __log2f(l_row)) * kLn2;
       const bool complete = pc.pa == 0 && pc.pe == sc.seq_start[b + 1] - sc.seq_start[b];
       float* obase;
       float* lbase;
@@ -651,7 +714,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       it += n;
       ++piece;
     }
-    if (sender) bulk_wait_all();  // our copies into the peer have landed
   }
 
   // ------------------------------------------------------------ teardown

@@ -92,6 +92,33 @@ def test_poison_never_reaches_output():
     assert_close(out, lse, *oracle_for(case), "poison")
 
 
+@pytest.mark.parametrize("scale", [0.0, -0.0625, 0.5])
+def test_softmax_scale_zero_negative_large(scale):
+    """A zero scale gives uniform weights, a negative one flips the ranking, a large
+    one makes the running maximum jump several times within a sequence."""
+    case = S.make_decode_case(4, 128, [1, 63, 700, 2000], seed=45, poison=True, softmax_scale=scale)
+    out, lse, err = run_decode(case)
+    assert err == 0
+    assert_close(out, lse, *oracle_for(case), f"scale {scale}")
+
+
+def test_growing_scores_force_rescales():
+    """The rope dims grow along the sequence (factor 1 + 40 t / T): they enter the
+    scores but not V, so the running maximum rises 3-9 times per head (by more than
+    the lazy-rescale threshold each time) while the values keep their size."""
+    lens = [640, 2000, 4100]
+    case = S.make_decode_case(3, 128, lens, seed=46, poison=True)
+    kv = S.bf16_bits_to_f32(case.kv_cache)
+    for b, T in enumerate(lens):
+        for t in range(T):
+            pg, r = case.block_table[b, t // 64], t % 64
+            kv[pg, r, 512:] *= 1.0 + 40.0 * t / T
+    case.kv_cache = S.f32_to_bf16_bits(kv)
+    out, lse, err = run_decode(case)
+    assert err == 0
+    assert_close(out, lse, *oracle_for(case), "growing scores")
+
+
 @pytest.mark.parametrize("workers", [1, 2, 7, 64, 148])
 def test_forced_split_counts_and_paged_equals_contiguous(workers):
     lens = [3000, 65, 1, 2048, 777]
