@@ -20,9 +20,10 @@
 // Pipeline.  The exchange has a long latency, so the softmax threads are software
 // pipelined: in each iteration they first send page j+1's partial (stage A) and
 // then finish page j (stage B), whose partial was sent one iteration earlier.  A
-// receive buffer is handed back to the peer as soon as it has been read.  P is
-// written (bf16) to shared memory and read from there by the PV MMA, which frees
-// each S buffer as soon as it has been loaded, so score MMAs run ahead.
+// receive buffer is handed back to the peer as soon as it has been read.  S is
+// freed as soon as the softmax has loaded it (stage A), so the score MMA of the
+// next page runs while the softmax finishes this one; P (bf16) goes to TMEM and
+// is the A operand of the PV MMA.
 //
 // Roles (384 threads): warp 0 issues TMA loads (and L2 prefetches a few pages
 // ahead), warp 1 allocates TMEM and issues MMAs (whichever of the next score MMA
@@ -34,12 +35,12 @@
 // exchange partial scores, run the online softmax (log2 domain, lazy rescale by at
 // most 2^8), write P, rescale O when needed, and write the epilogue.
 //
-// TMEM (512 columns): O [0,256) fp32, S double buffer [256,320) [320,384) fp32,
-// q' latent half [384,512) as bf16 pairs (the A operand of the latent QK^T).
+// TMEM (512 columns): O [0,256) fp32; q' (this CTA's 256 latent + 32 rope dims)
+// [256,400) as bf16 pairs, the A operand of QK^T; S [400,464) fp32; P [464,496) as
+// bf16 pairs, the A operand of PV.
 // Shared memory: 4 stages x (4 latent boxes [64 tokens x 64 dims], 128B swizzle:
 // K-major B of QK^T and MN-major B of PV; 1 rope box [64 tokens x 32 dims], 64B
-// swizzle); this CTA's rope part of q' [128 x 32] (64B swizzle, A operand); a 24 KB
-// send and a 24 KB receive buffer; a 16 KB P buffer (128B swizzle).
+// swizzle); a 24 KB send buffer and two 24 KB receive buffers.
 //
 // Every mbarrier wait is bounded by a time limit; on expiry the kernel records
 // MLA_ERR_DEVICE_TIMEOUT, tells the peer CTA to stop, drains its own TMA, bulk-copy
@@ -65,21 +66,20 @@ constexpr int kRopeBox = 64 * 64;                 // [64 rows x 32 bf16], 64B sw
 constexpr int kStageBytes = 4 * kLatBox + kRopeBox;  // 36864
 constexpr int kXRow = 64 * 3;                     // one head row of partial scores, 24 bits per value
 constexpr int kXBytes = 128 * kXRow;              // 24576: [128 heads x 64 tokens] partial scores
-constexpr int kPBytes = 128 * 128;                // [128 heads x 64 tokens] bf16 P
-constexpr int kSmemQRope = kStages * kStageBytes;             // 147456
-constexpr int kSmemTx = kSmemQRope + 128 * 64;                // 155648
-constexpr int kSmemRx = kSmemTx + kXBytes;                    // 180224: receive buffer
-constexpr int kSmemP = kSmemRx + kXBytes;                     // 204800: P (1024-aligned)
-constexpr int kSmemHmax = kSmemP + kPBytes;                   // 221184: half-row maxima [2][2][128]
+constexpr int kSmemTx = kStages * kStageBytes;                // 147456: send buffer
+constexpr int kSmemRx = kSmemTx + kXBytes;                    // 172032: 2 receive buffers
+constexpr int kSmemHmax = kSmemRx + 2 * kXBytes;              // 221184: half-row maxima [2][2][128]
 constexpr int kSmemLsum = kSmemHmax + 2 * 2 * 128 * 4;        // 223232: half-row sums [2][128]
 constexpr int kSmemBytes = kSmemLsum + 2 * 128 * 4;           // 224256
 constexpr int kSmemAlloc = kSmemBytes + 1024;                 // + alignment slack
 
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColO = 0, kColS = 256, kColQ = 384;
+// O fp32 [0,256); q' (latent 256 dims, then this CTA's 32 rope dims) as bf16 pairs
+// [256,400); S fp32 [400,464); P bf16 pairs [464,496).
+constexpr uint32_t kColO = 0, kColQ = 256, kColS = 400, kColP = 464;
 
-constexpr uint32_t kIdescQK = idesc_bf16_f32(128, 64, 0, 0);   // A K-major (TMEM or smem), B K-major
-constexpr uint32_t kIdescPV = idesc_bf16_f32(128, 256, 0, 1);  // A (P, smem) K-major, B MN-major
+constexpr uint32_t kIdescQK = idesc_bf16_f32(128, 64, 0, 0);   // A (q', TMEM), B K-major
+constexpr uint32_t kIdescPV = idesc_bf16_f32(128, 256, 0, 1);  // A (P, TMEM), B MN-major
 
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: P may reach 2^8 before O is rescaled
 constexpr int kPrefetch = 4;               // pages pulled into L2 ahead of the stage loads
@@ -89,11 +89,11 @@ enum Bar {
   kKvEmpty = kKvFull + kStages,
   kVReady = kKvEmpty + kStages,
   kSFull = kVReady + kStages,
-  kSFree = kSFull + 2,
-  kPFull = kSFree + 2,
-  kRxFull = kPFull + 1,
-  kPeerFree = kRxFull + 1,
-  kTxWritable = kPeerFree + 1,
+  kSFree = kSFull + 1,
+  kPFull = kSFree + 1,
+  kRxFull = kPFull + 1,     // [buffer]
+  kPeerFree = kRxFull + 2,  // [buffer]
+  kTxWritable = kPeerFree + 2,
   kTxReady = kTxWritable + 1,
   kXMax = kTxReady + 1,   // [page parity] half-row maxima published, receive buffer read
   kLSync = kXMax + 2,     // half-row sums published (epilogue)
@@ -143,9 +143,12 @@ struct Ctl {
   uint64_t limit_ns;
 };
 
-// Bounded wait on a local mbarrier phase; on timeout or abort returns false.  The
-// first probe is inline; only a wait that does not complete at once makes a call.
-__device__ __noinline__ bool wait_bar_slow(uint32_t bar, uint32_t parity, const Ctl& c) {
+// Bounded wait on a local mbarrier phase; on timeout or abort returns false.  Fully
+// inline (no call, so nothing is saved to the stack): try_wait suspends the thread
+// until the phase completes or a hardware time limit passes, and every 64 probes the
+// loop checks the abort flag and the time limit.
+__device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, const Ctl& c) {
+  if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = now_ns();
   for (uint32_t i = 1;; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
@@ -159,9 +162,6 @@ __device__ __noinline__ bool wait_bar_slow(uint32_t bar, uint32_t parity, const 
       }
     }
   }
-}
-__device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, const Ctl& c) {
-  return mbar_try_wait(bar, parity) || wait_bar_slow(bar, parity, c);
 }
 
 // Spin (bounded by time, ignoring the abort flag) until a phase completes: used only
@@ -186,7 +186,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
-  const uint32_t s_qrope = sbase + kSmemQRope, s_tx = sbase + kSmemTx, s_rx = sbase + kSmemRx, s_p = sbase + kSmemP;
+  const uint32_t s_tx = sbase + kSmemTx, s_rx = sbase + kSmemRx;
   auto bar = [&](int i) { return smem_u32(&bars[i]); };
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -204,13 +204,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       mbar_init(bar(kKvEmpty + s), 1);
       mbar_init(bar(kVReady + s), 1);
     }
-    for (int u = 0; u < 2; ++u) {
-      mbar_init(bar(kSFull + u), 1);      // MMA commit
-      mbar_init(bar(kSFree + u), 256);    // every softmax thread has loaded its half of S
-    }
+    mbar_init(bar(kSFull), 1);      // MMA commit
+    mbar_init(bar(kSFree), 256);    // every softmax thread has loaded its half of S
     mbar_init(bar(kPFull), 8);      // one arrival per softmax warp
-    mbar_init(bar(kRxFull), 1);     // armed (expect_tx) here, bytes from the peer
-    mbar_init(bar(kPeerFree), 1);   // the peer's receive buffer is read and re-armed
+    for (int u = 0; u < 2; ++u) {
+      mbar_init(bar(kRxFull + u), 1);     // armed (expect_tx) here, bytes from the peer
+      mbar_init(bar(kPeerFree + u), 1);   // the peer's receive buffer u is read and re-armed
+    }
     mbar_init(bar(kTxWritable), 1);
     mbar_init(bar(kTxReady), 8);
     for (int u = 0; u < 2; ++u) mbar_init(bar(kXMax + u), 8);
@@ -219,8 +219,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     mbar_init(bar(kOFull), 1);
     mbar_init(bar(kQReady), 256);
     mbar_init(bar(kDrain), 1);
-    // The receive buffer is armed for page 0 before the peer may send.
-    mbar_expect_tx(bar(kRxFull), kXBytes);
+    // Both receive buffers are armed (pages 0 and 1) before the peer may send.
+    mbar_expect_tx(bar(kRxFull + 0), kXBytes);
+    mbar_expect_tx(bar(kRxFull + 1), kXBytes);
     fence_mbar_init();
     tma_prefetch_desc(&kv_map);
     tma_prefetch_desc(&rope_map);
@@ -297,19 +298,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       int it = 0, piece = 0;
       bool ok = true;
       auto do_qk = [&](int g) {
-        const int s = g % kStages, u = g & 1;
+        const int s = g % kStages;
         tc_fence_after();
         const uint32_t kbase = sbase + s * kStageBytes;
-        const uint32_t d = tmem + kColS + 64 * u;
+        const uint32_t d = tmem + kColS;
 #pragma unroll
         for (int kc = 0; kc < 16; ++kc)
           mma_ts(d, tmem + kColQ + kc * 8, desc_sw128(kbase + (kc >> 2) * kLatBox + (kc & 3) * 32, 16, 1024),
                  kIdescQK, kc > 0 ? 1u : 0u);
 #pragma unroll
         for (int i = 0; i < 2; ++i)
-          mma_ss(d, desc_sw64(s_qrope + i * 32, 16, 512), desc_sw64(kbase + 4 * kLatBox + i * 32, 16, 512), kIdescQK,
-                 1u);
-        mma_commit(bar(kSFull + u));
+          mma_ts(d, tmem + kColQ + 128 + i * 8, desc_sw64(kbase + 4 * kLatBox + i * 32, 16, 512), kIdescQK, 1u);
+        mma_commit(bar(kSFull));
       };
       auto do_pv = [&](int g, bool first) {
         const int s = g % kStages;
@@ -317,8 +317,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         const uint32_t vbase = sbase + s * kStageBytes;
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
-          mma_ss(tmem + kColO, desc_sw128(s_p + kk * 32, 16, 1024), desc_sw128(vbase + kk * 2048, 8192, 1024),
-                 kIdescPV, (first && kk == 0) ? 0u : 1u);
+          mma_ts(tmem + kColO, tmem + kColP + kk * 8, desc_sw128(vbase + kk * 2048, 8192, 1024), kIdescPV,
+                 (first && kk == 0) ? 0u : 1u);
         mma_commit(bar(kKvEmpty + s));
         // The next completion of ODone after PV(g) is PV(g+1), which needs P(g+1),
         // which is written only after every softmax warp has seen PV(g) done.
@@ -330,7 +330,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       // softmax.  When neither is ready the thread sleeps on the next P (a bounded,
       // hinted try_wait), leaving the issue slots to the softmax warps.
       auto qk_ready = [&](int g) {
-        return (g < 2 || mbar_test(bar(kSFree + (g & 1)), ((g - 2) >> 1) & 1)) &&
+        return (g < 1 || mbar_test(bar(kSFree), (g - 1) & 1)) &&
                mbar_test(bar(kKvFull + g % kStages), (g / kStages) & 1);
       };
       auto pv_ready = [&](int g) {
@@ -413,14 +413,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(bar(kVReady + s));
-        // Every softmax warp has read the receive buffer (it published its half-row
-        // maxima after the read): re-arm it for page it+1 and let the peer send.  XMax
+        // Every softmax warp has read receive buffer u (it published its half-row
+        // maxima after the read): re-arm it for page it+2 and let the peer send.  XMax
         // is per page parity, so its next completion on this parity needs page it+2,
         // which the peer can only send after this: the wait cannot fall behind.
-        if (!__all_sync(0xffffffffu, wait_bar(bar(kXMax + (it & 1)), (it >> 1) & 1, ctl))) { ok = false; break; }
+        const int u = it & 1;
+        if (!__all_sync(0xffffffffu, wait_bar(bar(kXMax + u), (it >> 1) & 1, ctl))) { ok = false; break; }
         if (lane == 0) {
-          mbar_expect_tx(bar(kRxFull), kXBytes);
-          mbar_arrive_cluster(peer_free);
+          mbar_expect_tx(bar(kRxFull + u), kXBytes);
+          mbar_arrive_cluster(peer_free + u * 8);
         }
       }
     }
@@ -437,13 +438,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       bool ok = true;
       while (ok && pi.next(pc)) {
         for (int p = pc.pa; p < pc.pe; ++p, ++it) {
-          // All 8 softmax warps wrote their rows, and the peer has read page it-1 out of
-          // its receive buffer and re-armed it (the buffer starts armed for page 0).
-          if (!wait_bar(bar(kTxReady), it & 1, ctl) || (it > 0 && !wait_bar(bar(kPeerFree), (it - 1) & 1, ctl))) {
+          // All 8 softmax warps wrote their rows, and the peer has read page it-2 out of
+          // its receive buffer u and re-armed it (both buffers start armed).
+          const int u = it & 1, k = it >> 1;
+          if (!wait_bar(bar(kTxReady), it & 1, ctl) || !wait_bar(bar(kPeerFree + u), (k & 1) ^ 1, ctl)) {
             ok = false;
             break;
           }
-          bulk_copy_to_peer(rx_peer, s_tx, kXBytes, peer_rx_full);
+          bulk_copy_to_peer(rx_peer + u * kXBytes, s_tx, kXBytes, peer_rx_full + u * 8);
           bulk_wait_read_all();           // the copy has read the send buffer
           mbar_arrive(bar(kTxWritable));  // the softmax may write the next page into it
         }
@@ -464,6 +466,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     const uint32_t lane_off = (uint32_t)(32 * q) << 16;
     const uint32_t t_o = tmem + lane_off + kColO + 128 * wg;  // this thread's half of the O row
     const uint32_t t_q = tmem + lane_off + kColQ + 64 * wg;   // this thread's half of the q' latent columns
+    const uint32_t t_p = tmem + lane_off + kColP + 16 * wg;   // this thread's half of the P row
     // Scores stay unscaled (raw q'.k) until the exponent: a negative scale is moved
     // into q' as an exact sign flip, so max over raw scores is max over scaled ones
     // and each P costs one FFMA and one EX2.
@@ -483,14 +486,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     // Stage A of global page g: load this thread's half of the partial scores, free
     // the S buffer, and send them to the peer.
     auto stage_a = [&](int g, float (&own)[32]) -> bool {
-      const int u = g & 1, k = g >> 1;
-      if (!__all_sync(0xffffffffu, wait_bar(bar(kSFull + u), k & 1, ctl))) return false;
+      if (!__all_sync(0xffffffffu, wait_bar(bar(kSFull), g & 1, ctl))) return false;
       tc_fence_after();
       uint32_t r0[32];
-      tmem_ld32(tmem + lane_off + kColS + 64 * u + 32 * wg, r0);
+      tmem_ld32(tmem + lane_off + kColS + 32 * wg, r0);
       tmem_wait_ld();
       tc_fence_before();
-      mbar_arrive(bar(kSFree + u));
+      mbar_arrive(bar(kSFree));
 #pragma unroll
       for (int c = 0; c < 32; ++c) own[c] = __uint_as_float(r0[c]);
       // The previous page's copy out of the send buffer has finished reading it.
@@ -519,8 +521,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     while (ok && pi.next(pc)) {
       const int b = pc.b, n = pc.pe - pc.pa;
       const int T = a.seqlens[b];
-      // ---- stage q' for this sequence: latent half -> TMEM (split between the
-      // warpgroups), this CTA's 32 rope dims -> smem (64B swizzle)
+      // ---- stage q' for this sequence into TMEM: this CTA's latent half (split
+      // between the warpgroups) and its 32 rope dims
       {
         uint32_t qv[16];
         const bool live = row < a.heads;
@@ -537,20 +539,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           }
           tmem_st16(t_q + c * 16, qv);
         }
-        if (wg == 0) {
-          uint8_t* qr = smem + kSmemQRope + row * 64;
+        if (wg == 0) {  // this CTA's 32 rope dims: 16 columns after the latent ones
 #pragma unroll
-          for (int c = 0; c < 4; ++c) {  // 64B swizzle: 16-byte chunk c of row r at c ^ ((r >> 1) & 3)
-            uint4 v = live ? src[kDLatent / 8 + 4 * rank + c] : make_uint4(0, 0, 0, 0);
-            v.x ^= qsign;
-            v.y ^= qsign;
-            v.z ^= qsign;
-            v.w ^= qsign;
-            *reinterpret_cast<uint4*>(qr + ((c ^ ((row >> 1) & 3)) * 16)) = v;
+          for (int k = 0; k < 4; ++k) {
+            const uint4 v = live ? src[kDLatent / 8 + 4 * rank + k] : make_uint4(0, 0, 0, 0);
+            qv[4 * k + 0] = v.x ^ qsign;
+            qv[4 * k + 1] = v.y ^ qsign;
+            qv[4 * k + 2] = v.z ^ qsign;
+            qv[4 * k + 3] = v.w ^ qsign;
           }
+          tmem_st16(tmem + lane_off + kColQ + 128, qv);
         }
         tmem_wait_st();
-        fence_proxy_async();
         tc_fence_before();
         mbar_arrive(bar(kQReady));
       }
@@ -560,9 +560,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       // Stage B of page j of this piece: add the peer's partial, online softmax, write P.
       auto stage_b = [&](int j, float (&x)[32]) -> bool {
         const int g = it + j, u = g & 1, k = g >> 1, p = pc.pa + j;
-        if (!__all_sync(0xffffffffu, wait_bar(bar(kRxFull), g & 1, ctl))) return false;
+        if (!__all_sync(0xffffffffu, wait_bar(bar(kRxFull + u), k & 1, ctl))) return false;
         {
-          const uint8_t* rxrow = smem + kSmemRx + row * kXRow;
+          const uint8_t* rxrow = smem + kSmemRx + u * kXBytes + row * kXRow;
           uint32_t wd[24];
 #pragma unroll
           for (int c = 0; c < 6; ++c) {
@@ -597,9 +597,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int c = 0; c < 32; ++c) x[c] = c < valid ? x[c] : -INFINITY;
         }
-        float hm = x[0];
+        float mx[16];  // max is exact, so a tree (depth 5) gives the same value as a chain
 #pragma unroll
-        for (int c = 1; c < 32; ++c) hm = fmaxf(hm, x[c]);
+        for (int c = 0; c < 16; ++c) mx[c] = fmaxf(x[c], x[c + 16]);
+#pragma unroll
+        for (int w2 = 8; w2 >= 1; w2 >>= 1)
+#pragma unroll
+          for (int c = 0; c < w2; ++c) mx[c] = fmaxf(mx[c], mx[c + w2]);
+        const float hm = mx[0];
         hmax[(u * 2 + wg) * 128 + row] = hm;
         __syncwarp();
         if (lane == 0) mbar_arrive(bar(kXMax + u));
@@ -650,17 +655,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         uint32_t pk[16];
 #pragma unroll
         for (int c = 0; c < 16; ++c) pk[c] = pack_bf16x2(x[2 * c], x[2 * c + 1]);
-        // P [128 heads x 64 tokens] bf16, K-major, 128B swizzle (the PV A operand):
-        // this thread's 4 chunks of its row.  The buffer was last read by PV(g-1).
+        // P [128 heads x 64 tokens] as bf16 pairs in TMEM (the PV A operand): this
+        // thread's 16 columns of its row.  The columns were last read by PV(g-1).
         if (g >= 1 && !__all_sync(0xffffffffu, wait_bar(bar(kODone), (g - 1) & 1, ctl))) return false;
-        {
-          uint8_t* prow = smem + kSmemP + row * 128;
-#pragma unroll
-          for (int c = 0; c < 4; ++c)
-            *reinterpret_cast<uint4*>(prow + (((4 * wg + c) ^ (row & 7)) * 16)) =
-                make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
-        }
-        fence_proxy_async();
+        tc_fence_after();
+        tmem_st16(t_p, pk);
+        tmem_wait_st();
+        tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(bar(kPFull));
         return true;
