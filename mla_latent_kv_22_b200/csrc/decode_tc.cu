@@ -327,8 +327,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       // Issues whichever is ready first: the next score MMA (its S buffer freed and its
       // page loaded) or the next PV (its P written and its value rows cleaned), so score
       // MMAs run up to two pages ahead and never queue behind a PV that waits for the
-      // softmax.  When neither is ready the thread sleeps on the next P (a bounded,
-      // hinted try_wait), leaving the issue slots to the softmax warps.
+      // softmax.  When neither is ready the thread sleeps (a bounded, hinted try_wait)
+      // on the barrier of the next event: the next P, or the S buffer or page of the
+      // next score MMA, leaving the issue slots to the softmax warps.
       auto qk_ready = [&](int g) {
         return (g < 1 || mbar_test(bar(kSFree), (g - 1) & 1)) &&
                mbar_test(bar(kKvFull + g % kStages), (g / kStages) & 1);
@@ -361,7 +362,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             idle = 0;
             continue;
           }
-          if (gp < gq) mbar_try_wait_hint(bar(kPFull), gp & 1, 100);
+          if (gp < gq) {
+            mbar_try_wait_hint(bar(kPFull), gp & 1, 100);
+          } else if (gq >= 1 && !mbar_test(bar(kSFree), (gq - 1) & 1)) {  // next: QK(gq)
+            mbar_try_wait_hint(bar(kSFree), (gq - 1) & 1, 100);
+          } else {
+            mbar_try_wait_hint(bar(kKvFull + gq % kStages), (gq / kStages) & 1, 100);
+          }
           if ((++idle & 15) != 0) continue;
           if (abort_s) { ok = false; break; }
           const uint64_t t = now_ns();
@@ -481,7 +488,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     Piece pc;
     int it = 0, piece = 0;
     bool ok = true;
-    float own0[32], own1[32];
+    float cur[32], nxt[32];  // scores of the page being finished / of the next page
 
     // Stage A of global page g: load this thread's half of the partial scores, free
     // the S buffer, and send them to the peer.
@@ -586,7 +593,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           }
         }
         const int pid = pid_next;
-        if (j + 1 < n) pid_next = page_of(a, b, p + 1);  // used next page: latency off the chain
         if ((unsigned)pid >= (unsigned)np) {
           bad = true;
           set_device_error(a.err, MLA_ERR_DEVICE_BAD_PAGE);
@@ -608,6 +614,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         hmax[(u * 2 + wg) * 128 + row] = hm;
         __syncwarp();
         if (lane == 0) mbar_arrive(bar(kXMax + u));
+        // The next page's table entry is read here, right after a release (an arrive
+        // with release semantics waits for this thread's outstanding loads), so the
+        // read overlaps the exponentials and is back before the next release.
+        if (j + 1 < n) pid_next = page_of(a, b, p + 1);
         if (!__all_sync(0xffffffffu, wait_bar(bar(kXMax + u), k & 1, ctl))) return false;
         const float tmax = fmaxf(hm, hmax[(u * 2 + (wg ^ 1)) * 128 + row]);
         const float m_new = fmaxf(m, tmax);
@@ -666,14 +676,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         if (lane == 0) mbar_arrive(bar(kPFull));
         return true;
       };
-      ok = (it & 1) ? stage_a(it, own1) : stage_a(it, own0);
-      for (int j = 0; j < n && ok; ++j) {
-        const int g = it + j;
-        if (j + 1 < n) {
-          ok = (g & 1) ? stage_a(g + 1, own0) : stage_a(g + 1, own1);
-          if (!ok) break;
-        }
-        ok = (g & 1) ? stage_b(j, own1) : stage_b(j, own0);
+      // Step j sends page j's partial (stage A) and finishes page j-1 (stage B); each
+      // stage is inlined once and the register arrays rotate.
+      for (int j = 0; j <= n && ok; ++j) {
+        if (j < n && !(ok = stage_a(it + j, nxt))) break;
+        if (j > 0 && !(ok = stage_b(j - 1, cur))) break;
+#pragma unroll
+        for (int c = 0; c < 32; ++c) cur[c] = nxt[c];
       }
       if (!ok) break;
       // ---- epilogue: O / l (this thread's 128 of the CTA's 256 dims), lse
