@@ -143,21 +143,29 @@ struct Ctl {
   uint64_t limit_ns;
 };
 
-// Bounded wait on a local mbarrier phase; on timeout or abort returns false.  Fully
-// inline (no call, so nothing is saved to the stack): try_wait suspends the thread
-// until the phase completes or a hardware time limit passes, and every 64 probes the
-// loop checks the abort flag and the time limit.
+// Records a timed-out wait: the error word, this CTA's abort flag and the peer's.
+__device__ __noinline__ void wait_timed_out(int* err, volatile int* abort, uint32_t peer_abort) {
+  set_device_error(err, MLA_ERR_DEVICE_TIMEOUT);
+  *abort = 1;
+  asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(peer_abort), "r"(1) : "memory");
+}
+
+// Bounded wait on a local mbarrier phase; on timeout or abort returns false.  Inline
+// and small: try_wait suspends the thread until the phase completes or a hardware
+// time limit passes; only every 64th probe reads the abort flag and the global timer
+// (the start time is taken at the first such check), and the timeout itself is a call.
 __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, const Ctl& c) {
   if (mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = now_ns();
+  uint64_t t0 = 0;
   for (uint32_t i = 1;; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((i & 63) == 0) {
       if (*c.abort) return false;
-      if (now_ns() - t0 > c.limit_ns) {
-        set_device_error(c.err, MLA_ERR_DEVICE_TIMEOUT);
-        *c.abort = 1;
-        asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(c.peer_abort), "r"(1) : "memory");
+      const uint64_t t = now_ns();
+      if (t0 == 0) {
+        t0 = t;
+      } else if (t - t0 > c.limit_ns) {
+        wait_timed_out(c.err, c.abort, c.peer_abort);
         return false;
       }
     }
@@ -205,7 +213,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       mbar_init(bar(kVReady + s), 1);
     }
     mbar_init(bar(kSFull), 1);      // MMA commit
-    mbar_init(bar(kSFree), 256);    // every softmax thread has loaded its half of S
+    mbar_init(bar(kSFree), 8);      // every softmax warp has loaded its half of S
     mbar_init(bar(kPFull), 8);      // one arrival per softmax warp
     for (int u = 0; u < 2; ++u) {
       mbar_init(bar(kRxFull + u), 1);     // armed (expect_tx) here, bytes from the peer
@@ -217,7 +225,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     mbar_init(bar(kLSync), 8);
     mbar_init(bar(kODone), 1);
     mbar_init(bar(kOFull), 1);
-    mbar_init(bar(kQReady), 256);
+    mbar_init(bar(kQReady), 8);     // every softmax warp has staged its part of q'
     mbar_init(bar(kDrain), 1);
     // Both receive buffers are armed (pages 0 and 1) before the peer may send.
     mbar_expect_tx(bar(kRxFull + 0), kXBytes);
@@ -499,7 +507,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       tmem_ld32(tmem + lane_off + kColS + 32 * wg, r0);
       tmem_wait_ld();
       tc_fence_before();
-      mbar_arrive(bar(kSFree));
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(kSFree));  // one arrival per warp: 32 on one word would serialise
 #pragma unroll
       for (int c = 0; c < 32; ++c) own[c] = __uint_as_float(r0[c]);
       // The previous page's copy out of the send buffer has finished reading it.
@@ -559,7 +568,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         }
         tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(bar(kQReady));
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(kQReady));
       }
       float m = -INFINITY, l = 0.f;  // running max of raw scores, running sum
       bool bad = false;
