@@ -16,6 +16,7 @@ namespace {
 constexpr int kWarps = 4;
 
 __global__ void __launch_bounds__(kWarps * 32) combine_kernel(DecodeArgs a) {
+  grid_dep_wait();  // the decode grid's partials are complete and visible
   const int b = blockIdx.x;
   const int lane = threadIdx.x & 31;
   const int h = blockIdx.y * kWarps + (threadIdx.x >> 5);
@@ -72,8 +73,18 @@ __global__ void __launch_bounds__(kWarps * 32) combine_kernel(DecodeArgs a) {
 
 cudaError_t launch_combine(const DecodeArgs& a, cudaStream_t stream) {
   dim3 grid(a.batch, (a.heads + kWarps - 1) / kWarps);
-  combine_kernel<<<grid, kWarps * 32, 0, stream>>>(a);
-  return cudaGetLastError();
+  // Launched as a programmatic dependent of the decode grid: its launch overlaps
+  // the decode's tail, and grid_dep_wait() orders it after the decode's writes.
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(kWarps * 32, 1, 1);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, combine_kernel, a);
 }
 
 }  // namespace mla

@@ -242,6 +242,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   __syncthreads();
   cluster_sync();  // barriers of both CTAs initialised before any remote arrive
   tc_fence_after();
+  // Everything above overlaps the schedule grid; from here on its output is read.
+  grid_dep_wait();
   const uint32_t tmem = tmem_base_s;
   Ctl ctl{a.err, &abort_s, map_to_rank(smem_u32(&abort_s), peer), limit_ns};
 
@@ -737,6 +739,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   }
 
   // ------------------------------------------------------------ teardown
+  if (tid == 0) grid_dep_launch_dependents();  // the combine grid may launch (it waits for this grid's writes)
   tc_fence_before();
   __syncthreads();
   cluster_sync();  // the peer no longer writes into this CTA's shared memory
@@ -806,8 +809,19 @@ cudaError_t launch_decode_tc(const DecodeArgs& a, cudaStream_t stream) {
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
   const uint64_t limit_ns = (uint64_t)(a.wait_limit > 0 ? a.wait_limit : 1000) * 1000000ull;  // wait_limit in ms
-  decode_tc_kernel<<<2 * a.sched.num_workers, kThreads, kSmemAlloc, stream>>>(kv_map, rope_map, a, limit_ns);
-  return cudaGetLastError();
+  // Launched as a programmatic dependent of the schedule grid: the prologue (barrier
+  // set-up, TMEM allocation, descriptor prefetch) overlaps it.
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * a.sched.num_workers, 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = kSmemAlloc;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, decode_tc_kernel, kv_map, rope_map, a, limit_ns);
 }
 
 }  // namespace mla

@@ -79,6 +79,12 @@ __device__ __forceinline__ float2 unpack_f16x2(uint32_t v) {
   return __half22float2(h);
 }
 
+// Programmatic dependent launch: wait until the grid this one depends on has
+// completed and its writes are visible (a no-op when launched without the
+// attribute), and let this grid's dependents start launching.
+__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void grid_dep_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 __device__ __forceinline__ float fast_exp2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;\n" : "=f"(y) : "f"(x));

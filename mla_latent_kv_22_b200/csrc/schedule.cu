@@ -25,6 +25,7 @@ __global__ void __launch_bounds__(kSchedThreads) schedule_kernel(const int32_t* 
   __shared__ int warp_sums[kSchedThreads / 32];
   __shared__ int carry;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  grid_dep_launch_dependents();  // the decode grid may start its prologue now; it waits for this grid's writes
   if (tid == 0) carry = 0;
   __syncthreads();
 
