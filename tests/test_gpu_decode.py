@@ -133,6 +133,22 @@ def test_forced_split_counts_and_paged_equals_contiguous(workers):
     assert torch.equal(po, co) and torch.equal(pl, cl), "paged and contiguous differ"
 
 
+def test_two_piece_merge_deterministic_and_correct():
+    """Sequences split into two pieces are merged by whichever piece finishes last
+    (tcgen05 kernel); the result must not depend on which one that is.  Lengths of
+    15-17 pages over 16 workers give two- and three-piece sequences."""
+    lens = [1000, 1100, 900, 1024, 1030, 980, 1010, 1020]
+    case = S.make_decode_case(len(lens), 128, lens, seed=47)
+    M.mla_set_knob("num_workers", 16)
+    M.mla_set_knob("min_pages", 1)
+    dev = upload(case)
+    runs = [run_decode(case, dev) for _ in range(5)]
+    for o, l, e in runs:
+        assert e == 0
+        assert torch.equal(o, runs[0][0]) and torch.equal(l, runs[0][1])
+    assert_close(runs[0][0], runs[0][1], *oracle_for(case), "two-piece merge")
+
+
 def test_paged_equals_contiguous_default_and_shuffle_invariant():
     lens = S.uniform_seqlens(3, 16, 100, 3000)
     a = S.make_decode_case(16, 128, lens, seed=43, paged=True, shuffle=True)
