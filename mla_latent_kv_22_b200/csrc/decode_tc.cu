@@ -68,9 +68,7 @@ constexpr int kXRow = 64 * 3;                     // one head row of partial sco
 constexpr int kXBytes = 128 * kXRow;              // 24576: [128 heads x 64 tokens] partial scores
 constexpr int kSmemTx = kStages * kStageBytes;                // 147456: send buffer
 constexpr int kSmemRx = kSmemTx + kXBytes;                    // 172032: 2 receive buffers
-constexpr int kSmemHmax = kSmemRx + 2 * kXBytes;              // 221184: half-row maxima [2][2][128]
-constexpr int kSmemLsum = kSmemHmax + 2 * 2 * 128 * 4;        // 223232: half-row sums [2][128]
-constexpr int kSmemBytes = kSmemLsum + 2 * 128 * 4;           // 224256
+constexpr int kSmemBytes = kSmemRx + 2 * kXBytes;             // 221184
 constexpr int kSmemAlloc = kSmemBytes + 1024;                 // + alignment slack
 
 constexpr uint32_t kTmemCols = 512;
@@ -95,9 +93,8 @@ enum Bar {
   kPeerFree = kRxFull + 2,  // [buffer]
   kTxWritable = kPeerFree + 2,
   kTxReady = kTxWritable + 1,
-  kXMax = kTxReady + 1,   // [page parity] half-row maxima published, receive buffer read
-  kLSync = kXMax + 2,     // half-row sums published (epilogue)
-  kODone = kLSync + 1,    // PV(g) complete: O holds page g, P may be rewritten
+  kRxRead = kTxReady + 1,  // [page parity] every softmax warp has read receive buffer u
+  kODone = kRxRead + 2,    // PV(g) complete: O holds page g, P may be rewritten
   kOFull = kODone + 1,
   kQReady = kOFull + 1,
   kDrain = kQReady + 1,
@@ -221,8 +218,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     }
     mbar_init(bar(kTxWritable), 1);
     mbar_init(bar(kTxReady), 8);
-    for (int u = 0; u < 2; ++u) mbar_init(bar(kXMax + u), 8);
-    mbar_init(bar(kLSync), 8);
+    for (int u = 0; u < 2; ++u) mbar_init(bar(kRxRead + u), 8);
     mbar_init(bar(kODone), 1);
     mbar_init(bar(kOFull), 1);
     mbar_init(bar(kQReady), 8);     // every softmax warp has staged its part of q'
@@ -430,12 +426,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(bar(kVReady + s));
-        // Every softmax warp has read receive buffer u (it published its half-row
-        // maxima after the read): re-arm it for page it+2 and let the peer send.  XMax
-        // is per page parity, so its next completion on this parity needs page it+2,
-        // which the peer can only send after this: the wait cannot fall behind.
+        // Every softmax warp has read receive buffer u: re-arm it for page it+2 and let
+        // the peer send.  RxRead is per page parity, so its next completion on this
+        // parity needs page it+2, which the peer can only send after this: the wait
+        // cannot fall behind.
         const int u = it & 1;
-        if (!__all_sync(0xffffffffu, wait_bar(bar(kXMax + u), (it >> 1) & 1, ctl))) { ok = false; break; }
+        if (!__all_sync(0xffffffffu, wait_bar(bar(kRxRead + u), (it >> 1) & 1, ctl))) { ok = false; break; }
         if (lane == 0) {
           mbar_expect_tx(bar(kRxFull + u), kXBytes);
           mbar_arrive_cluster(peer_free + u * 8);
@@ -471,19 +467,24 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     }
     __syncwarp();
   } else if (warp >= 4) {
-    // ------------------------------------------------------------ softmax warpgroups
-    // Two warpgroups split every page's 64 score columns: warpgroup wg owns columns
-    // [32 wg, 32 wg + 32) of each head row (and the same half of its O columns); the
-    // two threads of a row exchange their half-row maxima through shared memory, so
-    // both apply the same running max.
+    // ------------------------------------------------------------ softmax warps
+    // Each softmax warp owns 16 head rows (TMEM lanes) of its lane quadrant and all 64
+    // score columns of every page.  In the 16x32bx2 access shape thread t holds row
+    // (t mod 16) and column half t / 16, so both halves of a row sit in one warp and
+    // their maxima and sums meet through one shuffle.
     const int sw = warp - 4;               // softmax warp 0..7
-    const int wg = sw >> 2;                // column half
+    const int wg = sw >> 2;                // which 16 lanes of the quadrant (and which half of q')
     const int q = warp & 3;                // lane quadrant of this warp
-    const int row = 32 * q + lane;         // head row = TMEM lane
-    const uint32_t lane_off = (uint32_t)(32 * q) << 16;
-    const uint32_t t_o = tmem + lane_off + kColO + 128 * wg;  // this thread's half of the O row
-    const uint32_t t_q = tmem + lane_off + kColQ + 64 * wg;   // this thread's half of the q' latent columns
-    const uint32_t t_p = tmem + lane_off + kColP + 16 * wg;   // this thread's half of the P row
+    const int ch = lane >> 4;              // column half of the row held by this thread
+    const int row = 32 * q + 16 * wg + (lane & 15);                 // head row = TMEM lane
+    const uint32_t lane_off = (uint32_t)(32 * q + 16 * wg) << 16;  // first of this warp's 16 lanes
+    const uint32_t t_o = tmem + lane_off + kColO;  // O rows: this thread's 128 columns start 128 ch on
+    const uint32_t t_p = tmem + lane_off + kColP;  // P rows: this thread's 16 columns start 16 ch on
+    // q' is staged with 32x32b stores (thread = lane of the quadrant); the two warps of
+    // a quadrant split its latent columns.
+    const int qrow = 32 * q + lane;
+    const uint32_t qlane_off = (uint32_t)(32 * q) << 16;
+    const uint32_t t_q = tmem + qlane_off + kColQ + 64 * wg;
     // Scores stay unscaled (raw q'.k) until the exponent: a negative scale is moved
     // into q' as an exact sign flip, so max over raw scores is max over scaled ones
     // and each P costs one FFMA and one EX2.
@@ -492,8 +493,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     const float thr_raw = scale2 > 0.f ? kRescaleThreshold / scale2 : INFINITY;
     uint8_t* txrow = smem + kSmemTx + row * kXRow;
     const int sw2 = (row >> 1) & 3;  // chunk swizzle of 192-byte rows: XOR keeps groups of 4 chunks
-    float* hmax = reinterpret_cast<float*>(smem + kSmemHmax);  // [page parity][wg][row]
-    float* lsum = reinterpret_cast<float*>(smem + kSmemLsum);  // [wg][row]
     PieceIter pi(sc, w);
     Piece pc;
     int it = 0, piece = 0;
@@ -506,7 +505,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       if (!__all_sync(0xffffffffu, wait_bar(bar(kSFull), g & 1, ctl))) return false;
       tc_fence_after();
       uint32_t r0[32];
-      tmem_ld32(tmem + lane_off + kColS + 32 * wg, r0);
+      tmem_ld16x2_32<32>(tmem + lane_off + kColS, r0);
       tmem_wait_ld();
       tc_fence_before();
       __syncwarp();
@@ -527,7 +526,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         }
 #pragma unroll
         for (int c = 0; c < 6; ++c)
-          *reinterpret_cast<uint4*>(txrow + (((6 * wg + c) ^ sw2) * 16)) =
+          *reinterpret_cast<uint4*>(txrow + (((6 * ch + c) ^ sw2) * 16)) =
               make_uint4(wd[4 * c], wd[4 * c + 1], wd[4 * c + 2], wd[4 * c + 3]);
       }
       fence_proxy_async();
@@ -543,8 +542,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       // between the warpgroups) and its 32 rope dims
       {
         uint32_t qv[16];
-        const bool live = row < a.heads;
-        const uint4* src = reinterpret_cast<const uint4*>(a.q + ((size_t)b * a.heads + (live ? row : 0)) * kDQK);
+        const bool live = qrow < a.heads;
+        const uint4* src = reinterpret_cast<const uint4*>(a.q + ((size_t)b * a.heads + (live ? qrow : 0)) * kDQK);
 #pragma unroll
         for (int c = 0; c < 4; ++c) {  // 4 x 32 dims of this warpgroup's 128 latent dims
 #pragma unroll
@@ -566,7 +565,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             qv[4 * k + 2] = v.z ^ qsign;
             qv[4 * k + 3] = v.w ^ qsign;
           }
-          tmem_st16(tmem + lane_off + kColQ + 128, qv);
+          tmem_st16(tmem + qlane_off + kColQ + 128, qv);
         }
         tmem_wait_st();
         tc_fence_before();
@@ -585,7 +584,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           uint32_t wd[24];
 #pragma unroll
           for (int c = 0; c < 6; ++c) {
-            const uint4 v = *reinterpret_cast<const uint4*>(rxrow + (((6 * wg + c) ^ sw2) * 16));
+            const uint4 v = *reinterpret_cast<const uint4*>(rxrow + (((6 * ch + c) ^ sw2) * 16));
             wd[4 * c] = v.x;
             wd[4 * c + 1] = v.y;
             wd[4 * c + 2] = v.z;
@@ -609,7 +608,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           bad = true;
           set_device_error(a.err, MLA_ERR_DEVICE_BAD_PAGE);
         }
-        const int valid = min(kPage, T - p * kPage) - 32 * wg;  // valid columns of this half
+        const int valid = min(kPage, T - p * kPage) - 32 * ch;  // valid columns of this half
         const bool ragged = valid < 32;                          // only a sequence's last page
         if (ragged) {
 #pragma unroll
@@ -622,16 +621,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         for (int w2 = 8; w2 >= 1; w2 >>= 1)
 #pragma unroll
           for (int c = 0; c < w2; ++c) mx[c] = fmaxf(mx[c], mx[c + w2]);
-        const float hm = mx[0];
-        hmax[(u * 2 + wg) * 128 + row] = hm;
+        const float hm = mx[0];  // depends on every value read from the receive buffer
         __syncwarp();
-        if (lane == 0) mbar_arrive(bar(kXMax + u));
+        if (lane == 0) mbar_arrive(bar(kRxRead + u));
         // The next page's table entry is read here, right after a release (an arrive
         // with release semantics waits for this thread's outstanding loads), so the
         // read overlaps the exponentials and is back before the next release.
         if (j + 1 < n) pid_next = page_of(a, b, p + 1);
-        if (!__all_sync(0xffffffffu, wait_bar(bar(kXMax + u), k & 1, ctl))) return false;
-        const float tmax = fmaxf(hm, hmax[(u * 2 + (wg ^ 1)) * 128 + row]);
+        const float tmax = fmaxf(hm, __shfl_xor_sync(0xffffffffu, hm, 16));
         const float m_new = fmaxf(m, tmax);
         const bool need = !(m_new <= m + thr_raw);  // also true while m is -inf
         const float alpha = !need ? 1.f : (m == -INFINITY ? 0.f : fast_exp2((m - m_new) * scale2));
@@ -643,7 +640,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 #pragma unroll 1
           for (int c = 0; c < 4; ++c) {
             uint32_t r[32];
-            tmem_ld32(t_o + c * 32, r);
+            tmem_ld16x2_32<128>(t_o + c * 32, r);
             tmem_wait_ld();
             uint32_t w0[16], w1[16];
 #pragma unroll
@@ -651,8 +648,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
               w0[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
               w1[e] = __float_as_uint(__uint_as_float(r[16 + e]) * alpha);
             }
-            tmem_st16(t_o + c * 32, w0);
-            tmem_st16(t_o + c * 32 + 16, w1);
+            tmem_st16x2_16<128>(t_o + c * 32, w0);
+            tmem_st16x2_16<128>(t_o + c * 32 + 16, w1);
           }
           tmem_wait_st();
           tc_fence_before();
@@ -681,7 +678,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         // thread's 16 columns of its row.  The columns were last read by PV(g-1).
         if (g >= 1 && !__all_sync(0xffffffffu, wait_bar(bar(kODone), (g - 1) & 1, ctl))) return false;
         tc_fence_after();
-        tmem_st16(t_p, pk);
+        tmem_st16x2_16<16>(t_p, pk);
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
@@ -700,11 +697,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       // ---- epilogue: O / l (this thread's 128 of the CTA's 256 dims), lse
       if (!__all_sync(0xffffffffu, wait_bar(bar(kOFull), piece & 1, ctl))) { ok = false; break; }
       tc_fence_after();
-      lsum[wg * 128 + row] = l;
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar(kLSync));
-      if (!__all_sync(0xffffffffu, wait_bar(bar(kLSync), piece & 1, ctl))) { ok = false; break; }
-      const float l_row = lsum[row] + lsum[128 + row];
+      const float l_row = l + __shfl_xor_sync(0xffffffffu, l, 16);
       const float inv = bad ? NAN : 1.f / l_row;
       const float lse_v = bad ? NAN : (m * scale2 + __log2f(l_row)) * kLn2;
       const bool complete = pc.pa == 0 && pc.pe == sc.seq_start[b + 1] - sc.seq_start[b];
@@ -721,17 +714,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 #pragma unroll 1
       for (int c = 0; c < 4; ++c) {
         uint32_t r[32];
-        tmem_ld32(t_o + c * 32, r);
+        tmem_ld16x2_32<128>(t_o + c * 32, r);
         tmem_wait_ld();
         if (row < a.heads) {
-          float4* dst = reinterpret_cast<float4*>(obase + (size_t)row * kDLatent + 256 * rank + 128 * wg + 32 * c);
+          float4* dst = reinterpret_cast<float4*>(obase + (size_t)row * kDLatent + 256 * rank + 128 * ch + 32 * c);
 #pragma unroll
           for (int e = 0; e < 8; ++e)
             dst[e] = make_float4(__uint_as_float(r[4 * e]) * inv, __uint_as_float(r[4 * e + 1]) * inv,
                                  __uint_as_float(r[4 * e + 2]) * inv, __uint_as_float(r[4 * e + 3]) * inv);
         }
       }
-      if (rank == 0 && wg == 0 && row < a.heads) lbase[row] = lse_v;
+      if (rank == 0 && ch == 0 && row < a.heads) lbase[row] = lse_v;
       tc_fence_before();
       it += n;
       ++piece;
