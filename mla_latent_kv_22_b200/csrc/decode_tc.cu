@@ -514,15 +514,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       for (int c = 0; c < 32; ++c) own[c] = __uint_as_float(r0[c]);
       // The previous page's copy out of the send buffer has finished reading it.
       if (!__all_sync(0xffffffffu, wait_bar(bar(kTxWritable), g & 1, ctl))) return false;
-      // Each value is sent as the top 3 bytes of its fp32 pattern; 4 values a, b, c, d
-      // travel as [a1 a2 a3 d1] [b1 b2 b3 d2] [c1 c2 c3 d3], 32 values = 6 chunks.
+      // Each value is sent as the top 3 bytes of its fp32 pattern: 4 values a, b, c, d
+      // travel as the words (low byte first) [d1 a1 a2 a3] [d2 b1 b2 b3] [d3 c1 c2 c3],
+      // i.e. a, b and c with their lowest byte replaced by one byte of d; 32 values
+      // are 6 chunks.
       {
         uint32_t wd[24];
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
-          wd[3 * e + 0] = __byte_perm(r0[4 * e + 0], r0[4 * e + 3], 0x5321);
-          wd[3 * e + 1] = __byte_perm(r0[4 * e + 1], r0[4 * e + 3], 0x6321);
-          wd[3 * e + 2] = __byte_perm(r0[4 * e + 2], r0[4 * e + 3], 0x7321);
+          wd[3 * e + 0] = __byte_perm(r0[4 * e + 0], r0[4 * e + 3], 0x3215);
+          wd[3 * e + 1] = __byte_perm(r0[4 * e + 1], r0[4 * e + 3], 0x3216);
+          wd[3 * e + 2] = __byte_perm(r0[4 * e + 2], r0[4 * e + 3], 0x3217);
         }
 #pragma unroll
         for (int c = 0; c < 6; ++c)
@@ -590,17 +592,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             wd[4 * c + 2] = v.z;
             wd[4 * c + 3] = v.w;
           }
-          // The dropped low byte is refilled with 0x80 (mid-point): relative error <= 2^-16.
-          constexpr uint32_t kMid = 0x80808080u;
+          // Each word read as an fp32 pattern is its value with the lowest mantissa
+          // byte replaced by another value's byte: relative error below 2^-15.  d is
+          // rebuilt as [d1 d1 d2 d3] (low byte first), with the same bound.
 #pragma unroll
           for (int e = 0; e < 8; ++e) {
             const uint32_t w0 = wd[3 * e], w1 = wd[3 * e + 1], w2 = wd[3 * e + 2];
-            x[4 * e + 0] += __uint_as_float(__byte_perm(w0, kMid, 0x2104));
-            x[4 * e + 1] += __uint_as_float(__byte_perm(w1, kMid, 0x2104));
-            x[4 * e + 2] += __uint_as_float(__byte_perm(w2, kMid, 0x2104));
-            const uint32_t t0 = __byte_perm(w0, kMid, 0x0034);  // [0x80, d1, -, -]
-            const uint32_t t1 = __byte_perm(w1, w2, 0x0073);    // [d2, d3, -, -]
-            x[4 * e + 3] += __uint_as_float(__byte_perm(t0, t1, 0x5410));
+            x[4 * e + 0] += __uint_as_float(w0);
+            x[4 * e + 1] += __uint_as_float(w1);
+            x[4 * e + 2] += __uint_as_float(w2);
+            const uint32_t t = __byte_perm(w0, w1, 0x4000);  // [d1 d1 d1 d2]
+            x[4 * e + 3] += __uint_as_float(__byte_perm(t, w2, 0x4310));
           }
         }
         const int pid = pid_next;
@@ -614,14 +616,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int c = 0; c < 32; ++c) x[c] = c < valid ? x[c] : -INFINITY;
         }
-        float mx[16];  // max is exact, so a tree (depth 5) gives the same value as a chain
+        // max is exact, so a tree of three-input maxima gives the same value as a chain
+        float m11[11];
 #pragma unroll
-        for (int c = 0; c < 16; ++c) mx[c] = fmaxf(x[c], x[c + 16]);
-#pragma unroll
-        for (int w2 = 8; w2 >= 1; w2 >>= 1)
-#pragma unroll
-          for (int c = 0; c < w2; ++c) mx[c] = fmaxf(mx[c], mx[c + w2]);
-        const float hm = mx[0];  // depends on every value read from the receive buffer
+        for (int c = 0; c < 10; ++c) m11[c] = fmax3(x[3 * c], x[3 * c + 1], x[3 * c + 2]);
+        m11[10] = fmaxf(x[30], x[31]);
+        const float hm = fmaxf(fmax3(fmax3(m11[0], m11[1], m11[2]), fmax3(m11[3], m11[4], m11[5]),
+                                     fmax3(m11[6], m11[7], m11[8])),
+                               fmaxf(m11[9], m11[10]));  // depends on every value read from the receive buffer
         __syncwarp();
         if (lane == 0) mbar_arrive(bar(kRxRead + u));
         // The next page's table entry is read here, right after a release (an arrive
