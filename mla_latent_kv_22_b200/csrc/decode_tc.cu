@@ -598,11 +598,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int e = 0; e < 8; ++e) {
             const uint32_t w0 = wd[3 * e], w1 = wd[3 * e + 1], w2 = wd[3 * e + 2];
-            x[4 * e + 0] += __uint_as_float(w0);
-            x[4 * e + 1] += __uint_as_float(w1);
-            x[4 * e + 2] += __uint_as_float(w2);
             const uint32_t t = __byte_perm(w0, w1, 0x4000);  // [d1 d1 d1 d2]
-            x[4 * e + 3] += __uint_as_float(__byte_perm(t, w2, 0x4310));
+            const float d = __uint_as_float(__byte_perm(t, w2, 0x4310));
+            const uint64_t s01 = f2_add(f2_pack(x[4 * e], x[4 * e + 1]), f2_pack(__uint_as_float(w0), __uint_as_float(w1)));
+            const uint64_t s23 = f2_add(f2_pack(x[4 * e + 2], x[4 * e + 3]), f2_pack(__uint_as_float(w2), d));
+            f2_unpack(s01, x[4 * e], x[4 * e + 1]);
+            f2_unpack(s23, x[4 * e + 2], x[4 * e + 3]);
           }
         }
         const int pid = pid_next;
@@ -658,20 +659,27 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         }
         l *= alpha;
         const float ms = m * scale2;
+        const uint64_t s2 = f2_pack(scale2, scale2), nms = f2_pack(-ms, -ms);
 #pragma unroll
-        for (int c = 0; c < 32; ++c) x[c] = fast_exp2(fmaf(x[c], scale2, -ms));
+        for (int c = 0; c < 32; c += 2) {
+          float y0, y1;
+          f2_unpack(f2_fma(f2_pack(x[c], x[c + 1]), s2, nms), y0, y1);
+          x[c] = fast_exp2(y0);
+          x[c + 1] = fast_exp2(y1);
+        }
         if (ragged) {  // a zero scale turns -inf into NaN above
 #pragma unroll
           for (int c = 0; c < 32; ++c) x[c] = c < valid ? x[c] : 0.f;
         }
-        float rs0 = 0.f, rs1 = 0.f, rs2 = 0.f, rs3 = 0.f;
+        uint64_t a01 = f2_pack(0.f, 0.f), a23 = a01;  // four running sums, two per instruction
 #pragma unroll
         for (int c = 0; c < 32; c += 4) {
-          rs0 += x[c];
-          rs1 += x[c + 1];
-          rs2 += x[c + 2];
-          rs3 += x[c + 3];
+          a01 = f2_add(a01, f2_pack(x[c], x[c + 1]));
+          a23 = f2_add(a23, f2_pack(x[c + 2], x[c + 3]));
         }
+        float rs0, rs1, rs2, rs3;
+        f2_unpack(a01, rs0, rs1);
+        f2_unpack(a23, rs2, rs3);
         l += (rs0 + rs1) + (rs2 + rs3);
         uint32_t pk[16];
 #pragma unroll
