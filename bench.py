@@ -22,6 +22,7 @@ import hashlib
 import json
 import math
 import os
+import re
 import statistics
 import sys
 import threading
@@ -62,16 +63,24 @@ def measured_peaks() -> tuple[dict, str]:
     return {"hbm_gbs": FALLBACK_HBM_GBS, "bf16_tflops": FALLBACK_BF16_TFLOPS}, "fallback"
 
 
+def strip_comments(src: str) -> str:
+    """C++ source without comments and blank space, so that editing a comment does not
+    count as changing the code (no string literal in these files contains //)."""
+    src = re.sub(r"/\*.*?\*/", " ", src, flags=re.S)
+    src = re.sub(r"//[^\n]*", " ", src)
+    return " ".join(src.split())
+
+
 def decode_source_hash(kernel: str) -> str:
-    """Hash of the sources of the decode kernel that ran (and the headers it uses),
-    to tie an ncu traffic figure to exactly that code."""
+    """Hash of the code of the decode kernel that ran (and the headers it uses), comments
+    and layout ignored, to tie an ncu traffic figure to exactly that code."""
     files = {"tcgen05": ["decode_tc.cu", "sm100_ptx.cuh"], "mma.sync": ["decode_mma.cu"]}[kernel]
     files += ["mla_device.cuh", "mla_internal.h"]
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "mla_latent_kv_22_b200", "csrc")
     for name in files:
-        with open(os.path.join(csrc, name), "rb") as f:
-            h.update(name.encode() + f.read())
+        with open(os.path.join(csrc, name), encoding="utf-8") as f:
+            h.update(name.encode() + strip_comments(f.read()).encode())
     return h.hexdigest()[:16]
 
 

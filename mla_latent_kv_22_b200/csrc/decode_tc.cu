@@ -11,8 +11,9 @@
 // loads only its part of every row (HBM and L2 traffic 1x), computes a partial S,
 // and the two partials are exchanged through distributed shared memory by bulk
 // copies and added.  Each exchanged score is the top 3 bytes of its fp32 pattern
-// (sign, exponent, 15 mantissa bits), the dropped byte refilled with its mid-point
-// (relative error <= 2^-16), 4 values in 12 bytes: 24 KB per page each way.  Each
+// (sign, exponent, 15 mantissa bits); on arrival its lowest byte holds a byte of
+// another value (relative error < 2^-15), 4 values in 12 bytes: 24 KB per page each
+// way.  Each
 // CTA adds its own exact partial to the peer's, so the two softmaxes agree to that
 // rounding; each CTA normalises its half of O by its own row sums, and rank 0
 // writes the lse.
@@ -29,11 +30,11 @@
 // ahead), warp 1 allocates TMEM and issues MMAs (whichever of the next score MMA
 // and the next PV is ready first), warp 2 zeroes value rows past the sequence end
 // before PV reads them and hands read receive buffers back to the peer, warp 3
-// copies each page's packed partial scores to the peer, and
-// warps 4..11 are two softmax warpgroups (one thread per
-// head row = TMEM lane, each warpgroup half of every page's columns) that stage q',
-// exchange partial scores, run the online softmax (log2 domain, lazy rescale by at
-// most 2^8), write P, rescale O when needed, and write the epilogue.
+// copies each page's packed partial scores to the peer, and warps 4..11 are the
+// softmax warps: each owns 16 head rows (TMEM lanes) and all 64 columns of every
+// page, both halves of a row in one warp (16x32bx2 TMEM access), and stages q',
+// exchanges partial scores, runs the online softmax (log2 domain, lazy rescale by
+// at most 2^8), writes P, rescales O when needed, and writes the epilogue.
 //
 // TMEM (512 columns): O [0,256) fp32; q' (this CTA's 256 latent + 32 rope dims)
 // [256,400) as bf16 pairs, the A operand of QK^T; S [400,464) fp32; P [464,496) as
@@ -541,13 +542,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       const int b = pc.b, n = pc.pe - pc.pa;
       const int T = a.seqlens[b];
       // ---- stage q' for this sequence into TMEM: this CTA's latent half (split
-      // between the warpgroups) and its 32 rope dims
+      // between the two warps of each lane quadrant) and its 32 rope dims
       {
         uint32_t qv[16];
         const bool live = qrow < a.heads;
         const uint4* src = reinterpret_cast<const uint4*>(a.q + ((size_t)b * a.heads + (live ? qrow : 0)) * kDQK);
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {  // 4 x 32 dims of this warpgroup's 128 latent dims
+        for (int c = 0; c < 4; ++c) {  // 4 x 32 dims of this warp's 128 latent dims
 #pragma unroll
           for (int k = 0; k < 4; ++k) {
             const uint4 v = live ? src[32 * rank + 16 * wg + 4 * c + k] : make_uint4(0, 0, 0, 0);
