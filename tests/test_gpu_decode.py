@@ -149,6 +149,25 @@ def test_two_piece_merge_deterministic_and_correct():
     assert_close(runs[0][0], runs[0][1], *oracle_for(case), "two-piece merge")
 
 
+def test_large_batch_crosses_schedule_passes():
+    """1,500 sequences (more than the schedule's 1,024-wide prefix-sum pass), lengths
+    0..200 with empty ones, few heads: every sequence's output against the oracle, and
+    the split counts 1 and 148 agree within rounding."""
+    lens = S.uniform_seqlens(48, 1500, 0, 200)
+    lens[::37] = 0
+    case = S.make_decode_case(1500, 8, lens, seed=48, poison=True)
+    dev = upload(case)
+    out, lse, err = run_decode(case, dev)
+    assert err == 0
+    assert_close(out, lse, *oracle_for(case), "B=1500")
+    for b in np.flatnonzero(lens == 0):
+        assert (out[b] == 0).all() and torch.isneginf(lse[b]).all()
+    M.mla_set_knob("num_workers", 1)
+    o1, l1, e1 = run_decode(case, dev)
+    assert e1 == 0
+    assert_close(o1, l1, *oracle_for(case), "B=1500, one worker")
+
+
 def test_paged_equals_contiguous_default_and_shuffle_invariant():
     lens = S.uniform_seqlens(3, 16, 100, 3000)
     a = S.make_decode_case(16, 128, lens, seed=43, paged=True, shuffle=True)
