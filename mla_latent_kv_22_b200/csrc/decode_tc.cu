@@ -13,10 +13,9 @@
 // copies and added.  Each exchanged score is the top 3 bytes of its fp32 pattern
 // (sign, exponent, 15 mantissa bits); on arrival its lowest byte holds a byte of
 // another value (relative error < 2^-15), 4 values in 12 bytes: 24 KB per page each
-// way.  Each
-// CTA adds its own exact partial to the peer's, so the two softmaxes agree to that
-// rounding; each CTA normalises its half of O by its own row sums, and rank 0
-// writes the lse.
+// way.  Each CTA adds its own exact partial to the peer's, so the two softmaxes agree
+// to that rounding; each CTA normalises its half of O by its own row sums, and rank
+// 0 writes the lse.
 //
 // Pipeline.  The exchange has a long latency, so the softmax threads are software
 // pipelined: in each iteration they first send page j+1's partial (stage A) and
