@@ -4,7 +4,9 @@
 //   L = ln sum_s e^{L_s},  out = sum_s e^{L_s - L} O_s
 // -- the rescaling the glossary's online-softmax note applies tile by tile, applied
 // once more across workers.  One warp per (sequence, head); each lane owns 16 of
-// the 512 dims as four float4 so every warp-wide load is 512 contiguous bytes.
+// the 512 dims as four float4 so every warp-wide load is 512 contiguous bytes.  The
+// partial slot of each piece comes from the sequence record (SeqInfo), so the loads
+// depend on one read only.
 // Sequences covered by a single worker were written by the decode kernel already;
 // empty sequences get out = 0, lse = -inf; invalid lengths get NaN.
 #include "mla_device.cuh"
@@ -32,15 +34,33 @@ __global__ void __launch_bounds__(kWarps * 32) combine_kernel(DecodeArgs a) {
     if (lane == 0) a.lse[(size_t)b * a.heads + h] = si.num_pieces == 0 ? -INFINITY : NAN;
     return;
   }
-  const int P = sc.num_workers;
-  const int q = *sc.quota;
-  const int st = sc.seq_start[b];
-  auto slot_of = [&](int k) {
-    const int w = si.first_worker + k;
-    return (w * q >= st) ? w : P + w;  // the piece is the worker's first sequence iff its range starts in b
+  const int np = si.num_pieces;
+  auto src_of = [&](int k) {
+    const int slot = k == 0 ? si.first_slot : si.first_worker + k;
+    return reinterpret_cast<const float4*>(sc.part_o + ((size_t)slot * a.heads + h) * kDLatent);
   };
-  float L = -INFINITY;
-  for (int k = lane; k < si.num_pieces; k += 32) L = fmaxf(L, sc.part_lse[(size_t)slot_of(k) * a.heads + h]);
+  auto lse_of = [&](int k) {
+    const int slot = k == 0 ? si.first_slot : si.first_worker + k;
+    return sc.part_lse[(size_t)slot * a.heads + h];
+  };
+  // The loads of the first kPre pieces (all that a sequence split in two needs) are
+  // issued together, right after the sequence record, so a warp waits for memory
+  // twice: lane k holds the lse of piece k and every lane its 16 dims of each piece's
+  // output.  Later pieces are loaded one by one.  The sums run in piece order either
+  // way.
+  constexpr int kPre = 2;
+  const float lk = lane < np ? lse_of(lane) : -INFINITY;
+  float4 v[kPre][4];
+#pragma unroll
+  for (int k = 0; k < kPre; ++k) {
+    if (k < np) {
+      const float4* src = src_of(k);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) v[k][i] = src[lane + 32 * i];
+    }
+  }
+  float L = lk;
+  for (int k = lane + 32; k < np; k += 32) L = fmaxf(L, lse_of(k));
 #pragma unroll
   for (int o = 16; o; o >>= 1) L = fmaxf(L, __shfl_xor_sync(0xffffffffu, L, o));
 
@@ -48,19 +68,25 @@ __global__ void __launch_bounds__(kWarps * 32) combine_kernel(DecodeArgs a) {
 #pragma unroll
   for (int i = 0; i < 4; ++i) acc[i] = make_float4(0.f, 0.f, 0.f, 0.f);
   float wsum = 0.f;
-  for (int k = 0; k < si.num_pieces; ++k) {
-    const int slot = slot_of(k);
-    const float wk = expf(sc.part_lse[(size_t)slot * a.heads + h] - L);
+  auto add = [&](float wk, const float4 (&x)[4]) {
     wsum += wk;
-    const float4* src = reinterpret_cast<const float4*>(sc.part_o + ((size_t)slot * a.heads + h) * kDLatent);
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      const float4 v = src[lane + 32 * i];
-      acc[i].x += wk * v.x;
-      acc[i].y += wk * v.y;
-      acc[i].z += wk * v.z;
-      acc[i].w += wk * v.w;
+      acc[i].x += wk * x[i].x;
+      acc[i].y += wk * x[i].y;
+      acc[i].z += wk * x[i].z;
+      acc[i].w += wk * x[i].w;
     }
+  };
+#pragma unroll
+  for (int k = 0; k < kPre; ++k)
+    if (k < np) add(expf(__shfl_sync(0xffffffffu, lk, k) - L), v[k]);
+  for (int k = kPre; k < np; ++k) {
+    const float4* src = src_of(k);
+    float4 x[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) x[i] = src[lane + 32 * i];
+    add(expf((k < 32 ? __shfl_sync(0xffffffffu, lk, k) : lse_of(k)) - L), x);
   }
   const float inv = 1.f / wsum;
 #pragma unroll

@@ -29,6 +29,7 @@ struct WorkerRange {
 struct SeqInfo {
   int first_worker;  // worker holding the sequence's first page
   int num_pieces;    // workers covering it; 0 = empty sequence; -1 = invalid length
+  int first_slot;    // partial slot of the first piece (piece k > 0 is in slot first_worker + k)
 };
 
 struct Schedule {

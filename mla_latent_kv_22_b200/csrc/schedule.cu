@@ -9,16 +9,6 @@ namespace {
 
 constexpr int kSchedThreads = 1024;
 
-// Largest b in [0, B) with start[b] <= g (start is non-decreasing, start[0] = 0).
-__device__ int seq_of_page(const int* start, int B, int g) {
-  int lo = 0, hi = B - 1;
-  while (lo < hi) {
-    int mid = (lo + hi + 1) >> 1;
-    if (start[mid] <= g) lo = mid; else hi = mid - 1;
-  }
-  return lo;
-}
-
 __global__ void __launch_bounds__(kSchedThreads) schedule_kernel(const int32_t* __restrict__ seqlens, int B,
                                                                  int max_blocks, int min_pages, Schedule s,
                                                                  int* err) {
@@ -29,15 +19,20 @@ __global__ void __launch_bounds__(kSchedThreads) schedule_kernel(const int32_t* 
   if (tid == 0) carry = 0;
   __syncthreads();
 
-  // 1. Exclusive prefix sum of pages per sequence, 1024 sequences per pass.
+  // 1. Exclusive prefix sum of pages per sequence, 1024 sequences per pass.  With a
+  // single pass, each thread keeps its sequence's start, page count and validity.
+  int my_start = 0, my_n = 0;
+  bool my_bad = false;
   for (int base = 0; base < B; base += kSchedThreads) {
     const int b = base + tid;
     int n = 0;
+    bool bad = false;
     if (b < B) {
       int T = seqlens[b];
       if (T < 0 || T > max_blocks * kPage) {
         set_device_error(err, MLA_ERR_DEVICE_BAD_PAGE);
         T = 0;  // the sequence is reported as invalid below; no page of it is read
+        bad = true;
       }
       n = (T + kPage - 1) / kPage;
     }
@@ -61,13 +56,15 @@ __global__ void __launch_bounds__(kSchedThreads) schedule_kernel(const int32_t* 
     __syncthreads();
     const int incl = x + (warp ? warp_sums[warp - 1] : 0) + carry;
     if (b < B) s.seq_start[b] = incl - n;
+    my_start = incl - n;
+    my_n = n;
+    my_bad = bad;
     __syncthreads();
     if (tid == kSchedThreads - 1) carry = incl;
     __syncthreads();
   }
   if (tid == 0) s.seq_start[B] = carry;
-  __threadfence_block();
-  __syncthreads();
+  if (B > kSchedThreads) __syncthreads();  // step 3 reloads seq_start[b + 1]
 
   const int N = carry;
   const int P = s.num_workers;
@@ -76,30 +73,45 @@ __global__ void __launch_bounds__(kSchedThreads) schedule_kernel(const int32_t* 
   if (q < 1) q = 1;
   if (tid == 0) *s.quota = q;
 
-  // 2. Worker ranges.
-  for (int w = tid; w < P; w += kSchedThreads) {
-    WorkerRange r{-1, 0, -1, 0};
-    const long long g0 = (long long)w * q;
-    if (g0 < N) {
-      const int g1 = (int)(g0 + q < (long long)N ? g0 + q : (long long)N);
-      r.b0 = seq_of_page(s.seq_start, B, (int)g0);
-      r.p0 = (int)g0 - s.seq_start[r.b0];
-      r.b1 = seq_of_page(s.seq_start, B, g1 - 1);
-      r.p1 = g1 - s.seq_start[r.b1];
-    }
-    s.ranges[w] = r;
-  }
+  // 2. Workers past the last page have no work.
+  for (int w = tid; w < P; w += kSchedThreads)
+    if ((long long)w * q >= N) s.ranges[w] = WorkerRange{-1, 0, -1, 0};
 
-  // 3. Per-sequence piece counts.
+  // 3. Per sequence: its piece count, and the range ends of the workers that overlap
+  // it.  Worker w covers pages [w q, min((w+1) q, N)); its first page lies in exactly
+  // one non-empty sequence, which writes (b0, p0), and so does its last page, which
+  // writes (b1, p1), so every field is written once and no search is needed.
   for (int b = tid; b < B; b += kSchedThreads) {
-    const int st = s.seq_start[b];
-    const int n = s.seq_start[b + 1] - st;
-    const int T = seqlens[b];
+    int st = my_start, n = my_n;
+    bool bad = my_bad;
+    if (B > kSchedThreads) {  // several passes: reload what this thread's pass computed
+      st = s.seq_start[b];
+      n = s.seq_start[b + 1] - st;
+      const int T = seqlens[b];
+      bad = T < 0 || T > max_blocks * kPage;
+    }
     SeqInfo si;
     si.first_worker = st / q;
     si.num_pieces = n > 0 ? (st + n - 1) / q - st / q + 1 : 0;
-    if (T < 0 || T > max_blocks * kPage) si.num_pieces = -1;
+    // The first piece is the worker's first sequence iff the worker's range starts at
+    // the sequence's first page; every later piece starts its worker's range.
+    si.first_slot = st % q == 0 ? si.first_worker : P + si.first_worker;
+    if (bad) si.num_pieces = -1;
     s.seq[b] = si;
+    if (n > 0) {
+      for (int w = st / q; w <= (st + n - 1) / q; ++w) {
+        const int g0 = w * q;
+        const int g1 = min(g0 + q, N);
+        if (g0 >= st) {
+          s.ranges[w].b0 = b;
+          s.ranges[w].p0 = g0 - st;
+        }
+        if (g1 <= st + n) {
+          s.ranges[w].b1 = b;
+          s.ranges[w].p1 = g1 - st;
+        }
+      }
+    }
   }
 }
 
