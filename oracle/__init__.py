@@ -30,6 +30,7 @@ from .mla_oracle import (  # noqa: F401
     bf16_to_f64,
     gather_rows,
     mla_decode_ref,
+    mla_decode_multi_ref,
     mla_decode_probs_ref,
     mla_decode_expanded_ref,
     mla_absorb_q_ref,

@@ -87,6 +87,41 @@ def mla_decode_ref(q, kv_cache, block_table, cache_seqlens, softmax_scale: float
     return out, lse
 
 
+def mla_decode_multi_ref(q, kv_cache, block_table, cache_seqlens, softmax_scale: float, *,
+                         d_v: int = 512, page_size: int = 64):
+    """Several new query tokens per sequence, each attending causally.
+
+    The pages define decode for one new token.  Reading taken for s_q > 1: the s_q new
+    tokens are the last s_q cached rows of sequence b, so query i (0 <= i < s_q) sits at
+    position T_b - s_q + i and attends to the rows t <= T_b - s_q + i, i.e. the first
+    n_i = T_b - s_q + 1 + i rows; over that window it is the single-token definition of
+    ``mla_decode_ref`` (scale on the whole 576-dim dot product, natural-log lse, values =
+    the first d_v dims of the rows).  An empty window (n_i <= 0) gives out = 0, lse = -inf.
+
+    q: [B, s_q, H, D].  Returns ``(out [B, s_q, H, d_v], lse [B, s_q, H])``.
+    """
+    B, SQ, H, _ = q.shape
+    out = np.zeros((B, SQ, H, d_v))
+    lse = np.full((B, SQ, H), -np.inf)
+    for b in range(B):
+        T = int(cache_seqlens[b])
+        if T <= 0:
+            continue
+        rows_all = gather_rows(kv_cache, block_table, b, T, page_size)   # [T, D]
+        for i in range(SQ):
+            n = T - SQ + 1 + i
+            if n <= 0:
+                continue
+            rows = rows_all[:n]
+            s = softmax_scale * (bf16_to_f64(q[b, i]) @ rows.T)          # [H, n]
+            m = s.max(axis=1, keepdims=True)
+            e = np.exp(s - m)
+            l = e.sum(axis=1, keepdims=True)
+            lse[b, i] = (m + np.log(l))[:, 0]
+            out[b, i] = (e / l) @ rows[:, :d_v]
+    return out, lse
+
+
 def mla_decode_probs_ref(q, kv_cache, block_table, cache_seqlens, softmax_scale: float, b: int, *,
                          page_size: int = 64) -> np.ndarray:
     """The softmax weights p[h, t] of sequence ``b`` (same definition as above)."""

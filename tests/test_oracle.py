@@ -17,7 +17,7 @@ import scipy.special
 import mla_synth as S
 import oracle as O
 from oracle import mla_oracle as OM
-from oracle.bruteforce import decode_bruteforce
+from oracle.bruteforce import decode_bruteforce, decode_multi_bruteforce
 
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "toy_expanded_vs_absorbed.txt")
 
@@ -250,6 +250,51 @@ def test_bruteforce_contiguous():
     bo, bl = decode_bruteforce(case.q, case.kv_cache, None, case.cache_seqlens, case.softmax_scale, 512)
     assert np.abs(out - np.array(bo)).max() <= 1e-13
     assert np.abs(lse - np.array(bl)).max() <= 1e-13
+
+
+# ---------------------------------------------------------------------------
+# 5b. Several causal query tokens per sequence (reading taken for s_q > 1).
+# ---------------------------------------------------------------------------
+
+def _multi_case(B, s_q, H, lens, seed, **kw):
+    """A decode case whose s_q * H query rows are viewed as [B, s_q, H, 576]."""
+    c = S.make_decode_case(B, s_q * H, lens, seed=seed, **kw)
+    return c, c.q.reshape(B, s_q, H, -1)
+
+
+def test_multi_query_bruteforce_with_explicit_mask():
+    # T = 2 with s_q = 3: query 0 sees nothing, query 1 token 0, query 2 tokens 0..1;
+    # T = 70 crosses a page boundary.  Brute force: loops, fsum, no max shift, and the
+    # causal mask written as t <= position.
+    c, q = _multi_case(2, 3, 2, [2, 70], seed=61, poison=True, latent_std=0.5)
+    out, lse = O.mla_decode_multi_ref(q, c.kv_cache, c.block_table, c.cache_seqlens, c.softmax_scale)
+    bo, bl = decode_multi_bruteforce(q, c.kv_cache, c.block_table, c.cache_seqlens, c.softmax_scale, 512)
+    bo, bl = np.array(bo), np.array(bl)
+    assert np.isneginf(lse[0, 0]).all() and (out[0, 0] == 0).all()
+    fin = np.isfinite(bl)
+    assert np.array_equal(fin, np.isfinite(lse))
+    assert np.abs(out - bo).max() <= 1e-13
+    assert np.abs(lse[fin] - bl[fin]).max() <= 1e-13
+
+
+def test_multi_query_windows_are_truncated_single_token_decodes():
+    # Query i of a sequence of length T is the single-token decode of the same cache cut
+    # to its first T - s_q + 1 + i tokens; the last query sees all T.
+    B, SQ, H = 3, 4, 2
+    lens = [5, 64, 131]
+    c, q = _multi_case(B, SQ, H, lens, seed=62, poison=True)
+    out, lse = O.mla_decode_multi_ref(q, c.kv_cache, c.block_table, c.cache_seqlens, c.softmax_scale)
+    for i in range(SQ):
+        cut = np.maximum(np.asarray(lens) - SQ + 1 + i, 0).astype(np.int32)
+        ro, rl = O.mla_decode_ref(q[:, i], c.kv_cache, c.block_table, cut, c.softmax_scale)
+        assert np.array_equal(out[:, i], ro) and np.array_equal(lse[:, i], rl)
+
+
+def test_multi_query_single_token_is_decode():
+    c, q = _multi_case(3, 1, 4, [1, 64, 300], seed=63, poison=True)
+    out, lse = O.mla_decode_multi_ref(q, c.kv_cache, c.block_table, c.cache_seqlens, c.softmax_scale)
+    ro, rl = O.mla_decode_ref(c.q, c.kv_cache, c.block_table, c.cache_seqlens, c.softmax_scale)
+    assert np.array_equal(out[:, 0], ro) and np.array_equal(lse[:, 0], rl)
 
 
 # ---------------------------------------------------------------------------
