@@ -105,6 +105,31 @@ mla_status_t mla_decode(const void* q, const void* kv_cache, const int32_t* bloc
                         float softmax_scale, mla_stream_t stream);
 
 /*
+ * mla_decode_multi -- mla_decode with s_q query tokens per sequence (multi-token
+ * prediction, speculative verification): the s_q new tokens are the last s_q
+ * cached rows of each sequence, and each attends causally.
+ *
+ * q       device bf16 [batch, s_q, heads, 576]
+ * out     device fp32 [batch, s_q, heads, 512], fully overwritten
+ * lse     device fp32 [batch, s_q, heads], fully overwritten
+ * Query i (0 <= i < s_q) of sequence b sits at position T_b - s_q + i and attends
+ * to the cached tokens t <= T_b - s_q + i, i.e. the first T_b - s_q + 1 + i rows;
+ * a query whose window is empty (T_b < s_q - i) gets out = 0, lse = -inf.  The
+ * pages describe single-token decode only; this is the causal reading of several
+ * new tokens appended to the cache before the call.  Each query row is computed as
+ * in mla_decode (s_q = 1 gives exactly mla_decode), with the s_q x heads rows of a
+ * sequence sharing every load of its cached rows.
+ * s_q >= 1 and s_q * heads <= 128, else MLA_ERR_UNSUPPORTED; it runs on the
+ * tcgen05 kernel only (MLA_ERR_UNSUPPORTED if the kernel knob forces the other).
+ * Every other argument, the workspace, determinism and error behaviour are those
+ * of mla_decode (mla_workspace_size takes s_q * heads as its heads).
+ */
+mla_status_t mla_decode_multi(const void* q, const void* kv_cache, const int32_t* block_table,
+                              const int32_t* cache_seqlens, float* out, float* lse,
+                              int batch, int s_q, int heads, int num_pages, int max_blocks,
+                              float softmax_scale, mla_stream_t stream);
+
+/*
  * mla_absorb_q -- key absorption, H independent GEMMs [batch x 128] x [128 x 512].
  *
  * q_nope  device bf16 [batch, heads, 128]

@@ -15,7 +15,7 @@ import os
 import torch
 
 __all__ = [
-    "MlaError", "mla_decode", "mla_decode_noalloc", "mla_absorb_q", "mla_absorb_o", "mla_workspace_size", "mla_set_workspace",
+    "MlaError", "mla_decode", "mla_decode_multi", "mla_decode_noalloc", "mla_absorb_q", "mla_absorb_o", "mla_workspace_size", "mla_set_workspace",
     "mla_get_device_error", "mla_status_string", "mla_set_knob", "mla_get_knob", "mla_selected_decode_kernel",
     "mla_timing_enable",
     "mla_timing_read", "lib", "LIB_PATH", "KNOB", "STATUS",
@@ -47,6 +47,7 @@ def _load() -> ctypes.CDLL:
     vp, i32, f32, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
     sig = {
         "mla_decode": ([vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, f32, vp], i32),
+        "mla_decode_multi": ([vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, f32, vp], i32),
         "mla_decode_noalloc": ([vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, f32, vp], i32),
         "mla_absorb_q": ([vp, vp, vp, vp, i32, i32, vp], i32),
         "mla_absorb_o": ([vp, vp, vp, i32, i32, vp], i32),
@@ -95,6 +96,21 @@ def _need(t: torch.Tensor, name: str, dtype: torch.dtype, shape: tuple | None = 
         raise ValueError(f"{name} must be contiguous")
 
 
+def _cache_args(kv_cache, block_table, B):
+    if block_table is None:
+        _need(kv_cache, "kv_cache", torch.bfloat16)
+        if kv_cache.dim() != 3 or kv_cache.shape[0] != B or kv_cache.shape[2] != D_QK or kv_cache.shape[1] % PAGE:
+            raise ValueError("contiguous kv_cache must be [B, Tcap, 576] with Tcap % 64 == 0")
+        return int(kv_cache.shape[1]) // PAGE, 0, None
+    _need(block_table, "block_table", torch.int32)
+    _need(kv_cache, "kv_cache", torch.bfloat16)
+    if kv_cache.dim() != 3 or tuple(kv_cache.shape[1:]) != (PAGE, D_QK):
+        raise ValueError("paged kv_cache must be [num_pages, 64, 576]")
+    if block_table.dim() != 2 or block_table.shape[0] != B:
+        raise ValueError("block_table must be [B, max_blocks]")
+    return int(block_table.shape[1]), int(kv_cache.shape[0]), block_table.data_ptr()
+
+
 def mla_decode(q, kv_cache, block_table, cache_seqlens, out, lse, softmax_scale: float, stream=None) -> None:
     """Absorbed decode (see include/mla.h).  q [B,H,576] bf16; kv_cache paged
     [num_pages,64,576] with block_table [B,max_blocks] int32, or contiguous
@@ -107,21 +123,26 @@ def mla_decode(q, kv_cache, block_table, cache_seqlens, out, lse, softmax_scale:
     _need(cache_seqlens, "cache_seqlens", torch.int32, (B,))
     _need(out, "out", torch.float32, (B, H, D_LATENT))
     _need(lse, "lse", torch.float32, (B, H))
-    if block_table is None:
-        _need(kv_cache, "kv_cache", torch.bfloat16)
-        if kv_cache.dim() != 3 or kv_cache.shape[0] != B or kv_cache.shape[2] != D_QK or kv_cache.shape[1] % PAGE:
-            raise ValueError("contiguous kv_cache must be [B, Tcap, 576] with Tcap % 64 == 0")
-        max_blocks, num_pages, bt = int(kv_cache.shape[1]) // PAGE, 0, None
-    else:
-        _need(block_table, "block_table", torch.int32)
-        _need(kv_cache, "kv_cache", torch.bfloat16)
-        if kv_cache.dim() != 3 or tuple(kv_cache.shape[1:]) != (PAGE, D_QK):
-            raise ValueError("paged kv_cache must be [num_pages, 64, 576]")
-        if block_table.dim() != 2 or block_table.shape[0] != B:
-            raise ValueError("block_table must be [B, max_blocks]")
-        max_blocks, num_pages, bt = int(block_table.shape[1]), int(kv_cache.shape[0]), block_table.data_ptr()
+    max_blocks, num_pages, bt = _cache_args(kv_cache, block_table, B)
     _check(lib.mla_decode(q.data_ptr(), kv_cache.data_ptr(), bt, cache_seqlens.data_ptr(), out.data_ptr(),
                           lse.data_ptr(), B, H, num_pages, max_blocks, float(softmax_scale), _stream(stream)))
+
+
+def mla_decode_multi(q, kv_cache, block_table, cache_seqlens, out, lse, softmax_scale: float, stream=None) -> None:
+    """Decode of s_q causal query tokens per sequence (see include/mla.h).
+    q [B,s_q,H,576] bf16; out [B,s_q,H,512] fp32; lse [B,s_q,H] fp32; the cache
+    arguments are those of mla_decode."""
+    if q.dim() != 4:
+        raise ValueError("q must be [B, s_q, H, 576]")
+    B, SQ, H = int(q.shape[0]), int(q.shape[1]), int(q.shape[2])
+    _need(q, "q", torch.bfloat16, (B, SQ, H, D_QK))
+    _need(cache_seqlens, "cache_seqlens", torch.int32, (B,))
+    _need(out, "out", torch.float32, (B, SQ, H, D_LATENT))
+    _need(lse, "lse", torch.float32, (B, SQ, H))
+    max_blocks, num_pages, bt = _cache_args(kv_cache, block_table, B)
+    _check(lib.mla_decode_multi(q.data_ptr(), kv_cache.data_ptr(), bt, cache_seqlens.data_ptr(), out.data_ptr(),
+                                lse.data_ptr(), B, SQ, H, num_pages, max_blocks, float(softmax_scale),
+                                _stream(stream)))
 
 
 def _noalloc_args(q, kv_cache, block_table, cache_seqlens, out, lse):

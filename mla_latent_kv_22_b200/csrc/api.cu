@@ -235,9 +235,16 @@ mla_status_t mla_get_device_error(mla_stream_t stream) {
   return v == MLA_ERR_DEVICE_TIMEOUT ? MLA_ERR_DEVICE_TIMEOUT : MLA_ERR_DEVICE_BAD_PAGE;
 }
 
-mla_status_t mla_decode(const void* q, const void* kv_cache, const int32_t* block_table,
-                        const int32_t* cache_seqlens, float* out, float* lse, int batch, int heads,
-                        int num_pages, int max_blocks, float softmax_scale, mla_stream_t stream_) {
+}  // extern "C"
+
+namespace mla {
+namespace {
+
+// mla_decode and mla_decode_multi: `heads` rows per sequence, made of s_q query
+// tokens of heads / s_q heads each.
+mla_status_t decode_call(const void* q, const void* kv_cache, const int32_t* block_table, const int32_t* cache_seqlens,
+                         float* out, float* lse, int batch, int s_q, int heads, int num_pages, int max_blocks,
+                         float softmax_scale, mla_stream_t stream_) {
   cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
   if (batch < 0 || heads < 0 || max_blocks < 0 || num_pages < 0)
     return fail(MLA_ERR_INVALID_ARG, "negative size (batch %d, heads %d, max_blocks %d, num_pages %d)", batch, heads,
@@ -263,6 +270,7 @@ mla_status_t mla_decode(const void* q, const void* kv_cache, const int32_t* bloc
   if (s != MLA_OK) return s;
   const int kernel = pick_kernel(heads);
   if (kernel < 0) return fail(MLA_ERR_UNSUPPORTED, "requested decode kernel does not handle heads = %d", heads);
+  if (s_q > 1 && kernel != 2) return fail(MLA_ERR_UNSUPPORTED, "several query tokens need the tcgen05 kernel");
   const int P = num_workers_for(*d, kernel, heads);
   const size_t need = carve_schedule(nullptr, batch, heads, P, nullptr);
   s = ensure_workspace(*d, need, stream);
@@ -284,6 +292,8 @@ mla_status_t mla_decode(const void* q, const void* kv_cache, const int32_t* bloc
   carve_schedule(d->ws, batch, heads, P, &a.sched);
   a.wait_limit = g_knobs[MLA_KNOB_WAIT_LIMIT].load() > 0 ? g_knobs[MLA_KNOB_WAIT_LIMIT].load() : 2000;  // ms
   a.withhold_arrive = g_knobs[MLA_KNOB_WITHHOLD_ARRIVE].load();
+  a.s_q = s_q;
+  a.hq = heads / s_q;
   const int min_pages = g_knobs[MLA_KNOB_MIN_PAGES].load() > 0 ? g_knobs[MLA_KNOB_MIN_PAGES].load() : 4;
 
   record_event(*d, 0, stream);
@@ -298,6 +308,28 @@ mla_status_t mla_decode(const void* q, const void* kv_cache, const int32_t* bloc
   record_event(*d, 3, stream);
   if (g_timing.load()) d->timed_calls++;
   return MLA_OK;
+}
+
+}  // namespace
+}  // namespace mla
+
+extern "C" {
+
+mla_status_t mla_decode(const void* q, const void* kv_cache, const int32_t* block_table,
+                        const int32_t* cache_seqlens, float* out, float* lse, int batch, int heads,
+                        int num_pages, int max_blocks, float softmax_scale, mla_stream_t stream) {
+  return decode_call(q, kv_cache, block_table, cache_seqlens, out, lse, batch, 1, heads, num_pages, max_blocks,
+                     softmax_scale, stream);
+}
+
+mla_status_t mla_decode_multi(const void* q, const void* kv_cache, const int32_t* block_table,
+                              const int32_t* cache_seqlens, float* out, float* lse, int batch, int s_q, int heads,
+                              int num_pages, int max_blocks, float softmax_scale, mla_stream_t stream) {
+  if (s_q < 1 || heads < 0) return fail(MLA_ERR_INVALID_ARG, "s_q = %d, heads = %d", s_q, heads);
+  if ((long long)s_q * heads > MLA_MAX_HEADS)
+    return fail(MLA_ERR_UNSUPPORTED, "s_q x heads = %lld rows > 128", (long long)s_q * heads);
+  return decode_call(q, kv_cache, block_table, cache_seqlens, out, lse, batch, s_q, s_q * heads, num_pages,
+                     max_blocks, softmax_scale, stream);
 }
 
 mla_status_t mla_absorb_q(const void* q_nope, const void* q_rope, const void* w_uk, void* q_out, int batch,

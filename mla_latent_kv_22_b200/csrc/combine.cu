@@ -63,6 +63,16 @@ __global__ void __launch_bounds__(kWarps * 32) combine_kernel(DecodeArgs a) {
   for (int k = lane + 32; k < np; k += 32) L = fmaxf(L, lse_of(k));
 #pragma unroll
   for (int o = 16; o; o >>= 1) L = fmaxf(L, __shfl_xor_sync(0xffffffffu, L, o));
+  if (L == -INFINITY) {
+    // No piece saw a token: a query row whose causal window is empty (several query
+    // tokens per sequence).  A NaN lse (a bad page) still makes the row NaN.
+    const bool nan = __any_sync(0xffffffffu, lk != lk);
+    const float v = nan ? NAN : 0.f;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) out4[lane + 32 * i] = make_float4(v, v, v, v);
+    if (lane == 0) a.lse[(size_t)b * a.heads + h] = nan ? NAN : -INFINITY;
+    return;
+  }
 
   float4 acc[4];
 #pragma unroll

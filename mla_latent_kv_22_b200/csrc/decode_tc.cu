@@ -181,6 +181,9 @@ __device__ __forceinline__ int page_of(const DecodeArgs& a, int b, int p) {
   return a.block_table ? a.block_table[(size_t)b * a.max_blocks + p] : b * a.max_blocks + p;
 }
 
+// kCausal: the rows of a sequence are several query tokens (DecodeArgs::s_q > 1),
+// each row masked to its query's window.
+template <bool kCausal>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     decode_tc_kernel(const __grid_constant__ CUtensorMap kv_map, const __grid_constant__ CUtensorMap rope_map,
                      const DecodeArgs a, uint64_t limit_ns) {
@@ -540,6 +543,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     while (ok && pi.next(pc)) {
       const int b = pc.b, n = pc.pe - pc.pa;
       const int T = a.seqlens[b];
+      // Tokens this row attends to: all T, or its query token's causal window.
+      const int Tq = kCausal && row < a.heads ? T - (a.s_q - 1 - row / a.hq) : T;
       // ---- stage q' for this sequence into TMEM: this CTA's latent half (split
       // between the two warps of each lane quadrant) and its 32 rope dims
       {
@@ -611,7 +616,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           bad = true;
           set_device_error(a.err, MLA_ERR_DEVICE_BAD_PAGE);
         }
-        const int valid = min(kPage, T - p * kPage) - 32 * ch;  // valid columns of this half
+        const int valid = min(kPage, Tq - p * kPage) - 32 * ch;  // valid columns of this half
         const bool ragged = valid < 32;                          // only a sequence's last page
         if (ragged) {
 #pragma unroll
@@ -708,8 +713,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       if (!__all_sync(0xffffffffu, wait_bar(bar(kOFull), piece & 1, ctl))) { ok = false; break; }
       tc_fence_after();
       const float l_row = l + __shfl_xor_sync(0xffffffffu, l, 16);
-      const float inv = bad ? NAN : 1.f / l_row;
-      const float lse_v = bad ? NAN : (m * scale2 + __log2f(l_row)) * kLn2;
+      // A causal row can see no token of a piece (or of its sequence): out 0, lse -inf.
+      const bool none = kCausal && l_row == 0.f;
+      const float inv = bad ? NAN : (none ? 0.f : 1.f / l_row);
+      const float lse_v = bad ? NAN : (none ? -INFINITY : (m * scale2 + __log2f(l_row)) * kLn2);
       const bool complete = pc.pa == 0 && pc.pe == sc.seq_start[b + 1] - sc.seq_start[b];
       float* obase;
       float* lbase;
@@ -776,9 +783,9 @@ int decode_tc_max_workers(int sm_count) {
     cfg.gridDim = dim3(2 * (sm_count / 2), 1, 1);
     cfg.blockDim = dim3(kThreads, 1, 1);
     cfg.dynamicSmemBytes = kSmemAlloc;
-    cudaFuncSetAttribute(decode_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemAlloc);
+    cudaFuncSetAttribute(decode_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemAlloc);
     int clusters = 0;
-    if (cudaOccupancyMaxActiveClusters(&clusters, decode_tc_kernel, &cfg) != cudaSuccess || clusters <= 0)
+    if (cudaOccupancyMaxActiveClusters(&clusters, decode_tc_kernel<false>, &cfg) != cudaSuccess || clusters <= 0)
       clusters = sm_count / 2;
     cached = clusters;
   }
@@ -788,7 +795,9 @@ int decode_tc_max_workers(int sm_count) {
 cudaError_t launch_decode_tc(const DecodeArgs& a, cudaStream_t stream) {
   static bool attr_set = false;
   if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(decode_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemAlloc);
+    cudaError_t e = cudaFuncSetAttribute(decode_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemAlloc);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(decode_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemAlloc);
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
@@ -824,7 +833,8 @@ cudaError_t launch_decode_tc(const DecodeArgs& a, cudaStream_t stream) {
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, decode_tc_kernel, kv_map, rope_map, a, limit_ns);
+  return a.s_q > 1 ? cudaLaunchKernelEx(&cfg, decode_tc_kernel<true>, kv_map, rope_map, a, limit_ns)
+                   : cudaLaunchKernelEx(&cfg, decode_tc_kernel<false>, kv_map, rope_map, a, limit_ns);
 }
 
 }  // namespace mla

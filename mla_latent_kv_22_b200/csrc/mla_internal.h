@@ -58,6 +58,10 @@ struct DecodeArgs {
   Schedule sched;
   int wait_limit;       // bounded-wait time limit in milliseconds (tcgen05 kernel)
   int withhold_arrive;  // test hook (tcgen05 kernel)
+  // Several query tokens per sequence (tcgen05 kernel only): the `heads` rows of a
+  // sequence are s_q query tokens of hq heads each (row r = query r / hq), and query
+  // i sees the first T - s_q + 1 + i cached tokens.  s_q = 1, hq = heads otherwise.
+  int s_q, hq;
 };
 
 cudaError_t launch_schedule(const int32_t* seqlens, int batch, int max_blocks, int min_pages,

@@ -115,6 +115,8 @@ extern "C" mla_status_t mla_decode_noalloc(const void* q, const void* kv_cache, 
   const int wl = mla::knob_value(MLA_KNOB_WAIT_LIMIT);
   a.wait_limit = wl > 0 ? wl : 2000;
   a.withhold_arrive = 0;
+  a.s_q = 1;
+  a.hq = heads;
   const int mp = mla::knob_value(MLA_KNOB_MIN_PAGES);
   const int min_pages = mp > 0 ? mp : 4;
 
