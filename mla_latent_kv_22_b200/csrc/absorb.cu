@@ -1,218 +1,570 @@
-// Key and value absorption: H independent small GEMMs (warp-level tensor cores).
+// Key and value absorption on the 5th-generation tensor cores: per call, H small
+// GEMMs, each of one head's weights against the whole batch.
 //
 //   absorb_q:  q'[b,h,0:512] = q_nope[b,h,:] W_UK[h]   ([B x 128] x [128 x 512]),
 //              q'[b,h,512:576] = q_rope[b,h,:]
 //   absorb_o:  out[b,h,:] = bf16(out_latent[b,h,:]) W_UV[h]   ([B x 512] x [512 x 128])
 // (glossary entry, "why absorb in decode": q^C (W^UK)^T and (sum_t p_t c_t) W^UV.)
 //
-// Both are HBM-bound (about 1 GFLOP against tens of MB at the largest workload),
-// so they are written for streaming: absorb_q computes a 64 x 128 output tile of
-// one head per CTA, loading its operands in two halves of K so the first half's
-// MMAs overlap the second half's loads, and writes the tile through shared memory
-// as whole rows; absorb_o computes a 64 x 128 tile of one head per CTA, streaming
-// K = 512 through a three-stage cp.async ring (fp32 out_latent is rounded to bf16
-// as its fragments are read).  Operands sit in XOR-swizzled shared memory; the
-// MMAs are warp-level bf16 tensor-core instructions with fp32 accumulation.
+// Both are HBM-bound (about 1 GFLOP against tens of MB at the largest workload), so
+// they are written for streaming.  A work item is one head and a tile of up to 128
+// batch rows (the MMA's M; rows past the batch are zero-filled by TMA on load and
+// clipped by TMA on store); CTAs are persistent over items, one per SM.  Roles:
+// warps 0-3 own the 128 TMEM lanes (epilogue, and for absorb_o the fp32 -> bf16
+// conversion of A), warp 4 issues TMA loads, warp 5 allocates TMEM and issues the
+// MMAs.  The accumulator is double-buffered in TMEM, so one tile's epilogue runs
+// under the next tile's MMAs.  Every wait is bounded: on expiry the kernel records
+// MLA_ERR_DEVICE_TIMEOUT, lets in-flight copies and MMAs finish, frees TMEM and
+// returns.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
 #include "mla_device.cuh"
 #include "mla_internal.h"
+#include "sm100_ptx.cuh"
 
 namespace mla {
 namespace {
 
-constexpr int kThreads = 128;
-constexpr int kTileM = 64, kTileN = 128, kTileK = 128;
-constexpr int kChunks = kTileK * 2 / 16;  // 16 chunks of 16 B per 128-wide bf16 row
+using namespace sm100;
 
-__device__ __forceinline__ uint32_t swz16(int r, int c) { return (uint32_t)(r * kChunks + (c ^ (r & 7))) * 16u; }
+constexpr int kThreads = 192;
+constexpr int kRows = 128;                // batch rows per item (MMA M)
+constexpr int kBox = kRows * 128;         // one [128 rows x 128 B] 128B-swizzled TMA box: 16 KB
 
-// acc[16x128] += A[16 x 16 k] * B[16 k x 128] over k-steps [kc0, kc1) of 16, for
-// warp rows [16w, 16w+16).
-__device__ __forceinline__ void warp_tile_mma(float (&acc)[16][4], uint32_t a_s, uint32_t b_s, int warp, int lane,
-                                              int kc0, int kc1) {
-  const int a_row = warp * 16 + (lane & 15);
-  const int b_row = (lane & 7) + (((lane >> 3) & 1) << 3);
-#pragma unroll
-  for (int kc = kc0; kc < kc1; ++kc) {
-    uint32_t af[4];
-    ldmatrix_x4(af, a_s + swz16(a_row, kc * 2 + (lane >> 4)));
-#pragma unroll
-    for (int nn = 0; nn < kTileN / 16; ++nn) {
-      uint32_t bf[4];
-      ldmatrix_x4_trans(bf, b_s + swz16(kc * 16 + b_row, nn * 2 + (lane >> 4)));
-      mma_bf16_16816(acc[2 * nn], af, bf[0], bf[1]);
-      mma_bf16_16816(acc[2 * nn + 1], af, bf[2], bf[3]);
+// ---------------------------------------------------------------- helpers
+__device__ __forceinline__ uint64_t now_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+struct Guard {
+  int* err;
+  volatile int* abort;
+  uint64_t limit_ns;
+};
+
+// Bounded wait on an mbarrier phase; false on timeout (recorded) or abort.
+__device__ __forceinline__ bool wait_on(uint32_t bar, uint32_t parity, const Guard& g) {
+  if (mbar_try_wait(bar, parity)) return true;
+  uint64_t t0 = 0;
+  for (uint32_t i = 1;; ++i) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((i & 63) == 0) {
+      if (*g.abort) return false;
+      const uint64_t t = now_ns();
+      if (t0 == 0) {
+        t0 = t;
+      } else if (t - t0 > g.limit_ns) {
+        set_device_error(g.err, MLA_ERR_DEVICE_TIMEOUT);
+        *g.abort = 1;
+        return false;
+      }
     }
   }
 }
-
-// Stage rows [r0, r1) and 16-byte chunks [c0, c1) of a [rows x 128] bf16 block (row
-// stride in elements) into swizzled smem; rows >= valid_rows are zero-filled.
-__device__ __forceinline__ void stage_bf16(uint32_t dst, const __nv_bfloat16* src, size_t stride, int r0, int r1,
-                                           int c0, int c1, int valid_rows, const void* safe) {
-  const int nc = c1 - c0;
-  for (int i = threadIdx.x; i < (r1 - r0) * nc; i += kThreads) {
-    const int r = r0 + i / nc, c = c0 + i % nc;
-    const bool ok = r < valid_rows;
-    cp_async_16(dst + swz16(r, c), ok ? (const void*)(src + r * stride + c * 8) : safe, ok ? 16 : 0);
+__device__ __forceinline__ void drain_on(uint32_t bar, uint32_t parity, uint64_t limit_ns) {
+  const uint64_t t0 = now_ns();
+  while (!mbar_try_wait(bar, parity) && now_ns() - t0 < limit_ns) {
   }
 }
 
-__global__ void __launch_bounds__(kThreads) absorb_q_kernel(const __nv_bfloat16* __restrict__ q_nope,
-                                                            const __nv_bfloat16* __restrict__ q_rope,
-                                                            const __nv_bfloat16* __restrict__ w_uk,
-                                                            __nv_bfloat16* __restrict__ q_out, int B, int H) {
-  __shared__ __align__(128) uint8_t a_tile[kTileM * kTileK * 2];
-  __shared__ __align__(128) uint8_t b_tile[kTileK * kTileN * 2];
-  const int b0 = blockIdx.x * kTileM, n0 = blockIdx.y * kTileN, h = blockIdx.z;
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int rows = min(kTileM, B - b0);
-  const __nv_bfloat16* a_src = q_nope + ((size_t)b0 * H + h) * MLA_D_NOPE;
-  const __nv_bfloat16* b_src = w_uk + (size_t)h * MLA_D_NOPE * kDLatent + n0;
-  // K in two halves: k [0,64) is A chunks [0,8) and B rows [0,64).
-#pragma unroll
-  for (int half = 0; half < 2; ++half) {
-    stage_bf16(smem_u32(a_tile), a_src, (size_t)H * MLA_D_NOPE, 0, kTileM, 8 * half, 8 * half + 8, rows, q_nope);
-    stage_bf16(smem_u32(b_tile), b_src, kDLatent, 64 * half, 64 * half + 64, 0, kChunks, kTileK, w_uk);
-    cp_async_commit();
-  }
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const void* map, int x, int y, int z, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cta.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(
+          dst),
+      "l"(map), "r"(x), "r"(y), "r"(z), "r"(bar)
+      : "memory");
+}
+// Tiled store of one box from shared memory (coordinates are never negative here).
+__device__ __forceinline__ void tma_store_3d(const void* map, uint32_t src, int x, int y, int z) {
+  asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%1, %2, %3}], [%4];" ::"l"(map), "r"(x),
+               "r"(y), "r"(z), "r"(src)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// At most one committed bulk group still reading shared memory.
+__device__ __forceinline__ void bulk_wait_read_1() { asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory"); }
+__device__ __forceinline__ void bar_sync_epilogue() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
 
-  float acc[16][4];
-#pragma unroll
-  for (int i = 0; i < 16; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.f;
-  cp_async_wait<1>();
-  __syncthreads();
-  warp_tile_mma(acc, smem_u32(a_tile), smem_u32(b_tile), warp, lane, 0, 4);
-  cp_async_wait<0>();
-  __syncthreads();
-  warp_tile_mma(acc, smem_u32(a_tile), smem_u32(b_tile), warp, lane, 4, 8);
-  __syncthreads();  // every warp is done with a_tile: it now holds the bf16 output tile
-
-  // Output tile [64 rows x 128 dims] bf16 through shared memory, then whole 256-byte
-  // row segments to global memory.
-  const int g = lane >> 2, t4 = lane & 3;
-#pragma unroll
-  for (int r = 0; r < 2; ++r) {
-    const int row = warp * 16 + g + r * 8;
-#pragma unroll
-    for (int i = 0; i < 16; ++i)  // columns 8i + 2 t4, +1: chunk i, word t4
-      *reinterpret_cast<uint32_t*>(a_tile + swz16(row, i) + t4 * 4) = pack_bf16x2(acc[i][2 * r], acc[i][2 * r + 1]);
-  }
-  __syncthreads();
-  for (int i = threadIdx.x; i < rows * kChunks; i += kThreads) {
-    const int r = i / kChunks, c = i % kChunks;
-    *reinterpret_cast<uint4*>(q_out + ((size_t)(b0 + r) * H + h) * kDQK + n0 + c * 8) =
-        *reinterpret_cast<const uint4*>(a_tile + swz16(r, c));
-  }
-  if (blockIdx.y == 0) {  // rope half of q' is a copy
-    for (int i = threadIdx.x; i < rows * 8; i += kThreads) {
-      const int r = i >> 3, c = i & 7;
-      const uint4 v = *reinterpret_cast<const uint4*>(q_rope + ((size_t)(b0 + r) * H + h) * kDRope + c * 8);
-      *reinterpret_cast<uint4*>(q_out + ((size_t)(b0 + r) * H + h) * kDQK + kDLatent + c * 8) = v;
-    }
-  }
+// 32 fp32 -> 16-byte chunks [q4] of bf16 (8 values each).
+__device__ __forceinline__ uint4 pack8(const uint32_t* v) {
+  return make_uint4(pack_bf16x2(__uint_as_float(v[0]), __uint_as_float(v[1])),
+                    pack_bf16x2(__uint_as_float(v[2]), __uint_as_float(v[3])),
+                    pack_bf16x2(__uint_as_float(v[4]), __uint_as_float(v[5])),
+                    pack_bf16x2(__uint_as_float(v[6]), __uint_as_float(v[7])));
 }
 
-constexpr int kOKc = 64;                                  // K per stage
-constexpr int kOStages = 3;
-constexpr int kOABytes = kTileM * kOKc * 4;               // fp32 A chunk [64 rows x 64 k]
-constexpr int kOStageBytes = kOABytes + kOKc * kTileN * 2;  // + bf16 B chunk [64 k x 128 n]
-constexpr int kOSmem = kOStages * kOStageBytes;           // 96 KB
+// ================================================================ absorb_q
+// Item (head h, batch tile mt): A = q_nope[128 rows x 128 k] (two K-major boxes), then
+// four n-tiles of 128: B = W_UK[h][128 k x 128 n] (two MN-major boxes), D = 128 x 128
+// fp32 in TMEM, written out as bf16 through shared memory by TMA stores.
+constexpr int kQA = 2 * kBox, kQB = 2 * kBox, kQO = 2 * kBox;  // 32 KB each
+constexpr int kQBStages = 4;             // every n-tile of an item's weights in flight at once
+constexpr int kQSmA = 0, kQSmB = kQA, kQSmO = kQSmB + kQBStages * kQB;
+constexpr int kQSmem = kQSmO + 2 * kQO;  // 224 KB: A, B[4], out[2]
+constexpr int kQNt = kDLatent / 128;     // n-tiles per item
+constexpr uint32_t kQIdesc = idesc_bf16_f32(128, 128, 0, 1);
 
-__global__ void __launch_bounds__(kThreads) absorb_o_kernel(const float* __restrict__ out_latent,
-                                                            const __nv_bfloat16* __restrict__ w_uv,
-                                                            float* __restrict__ out, int B, int H) {
-  extern __shared__ __align__(1024) uint8_t smem_o[];
-  const int b0 = blockIdx.x * kTileM, h = blockIdx.y;
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int rows = min(kTileM, B - b0);
-  const uint32_t sb = smem_u32(smem_o);
-  // Stage s <- K chunk kc: A rows of 64 fp32 (16 chunks of 16 B, chunk c of row r at
-  // c ^ (r & 7)), B rows of 128 bf16 in the same swizzle.
-  auto load = [&](int kc, int s) {
-    const uint32_t a_s = sb + s * kOStageBytes, b_s = a_s + kOABytes;
-    const int k0 = kc * kOKc;
-    for (int i = threadIdx.x; i < kTileM * 16; i += kThreads) {
-      const int r = i >> 4, c = i & 15;
-      const bool ok = r < rows;
-      cp_async_16(a_s + r * 256 + ((c ^ (r & 7)) * 16),
-                  ok ? (const void*)(out_latent + ((size_t)(b0 + r) * H + h) * kDLatent + k0 + c * 4) : out_latent,
-                  ok ? 16 : 0);
+enum QBar { kQAFull = 0, kQAEmpty, kQBFull, kQBEmpty = kQBFull + kQBStages, kQDFull = kQBEmpty + kQBStages, kQDEmpty = kQDFull + 2, kQDone = kQDEmpty + 2, kQNumBars };
+
+__global__ void __launch_bounds__(kThreads, 1)
+    absorb_q_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
+                       const __grid_constant__ CUtensorMap map_o, const __nv_bfloat16* __restrict__ q_rope,
+                       __nv_bfloat16* __restrict__ q_out, int B, int H, int* err, uint64_t limit_ns) {
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ __align__(8) uint64_t bars[kQNumBars];
+  __shared__ uint32_t tmem_s;
+  __shared__ int abort_s;
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  auto bar = [&](int i) { return smem_u32(&bars[i]); };
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int mtiles = (B + kRows - 1) / kRows;
+  const int items = H * mtiles;
+
+  if (tid == 0) {
+    abort_s = 0;
+    mbar_init(bar(kQAFull), 1);
+    mbar_init(bar(kQAEmpty), 1);
+    for (int i = 0; i < kQBStages; ++i) {
+      mbar_init(bar(kQBFull + i), 1);
+      mbar_init(bar(kQBEmpty + i), 1);
     }
-    for (int i = threadIdx.x; i < kOKc * 16; i += kThreads) {
-      const int r = i >> 4, c = i & 15;
-      cp_async_16(b_s + swz16(r, c), w_uv + ((size_t)h * kDLatent + k0 + r) * MLA_D_V + c * 8, 16);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(bar(kQDFull + i), 1);
+      mbar_init(bar(kQDEmpty + i), 4);  // one arrival per epilogue warp
     }
-  };
-  float acc[16][4];
-#pragma unroll
-  for (int i = 0; i < 16; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.f;
-  constexpr int kNk = kDLatent / kOKc;  // 8 chunks
-  load(0, 0);
-  cp_async_commit();
-  load(1, 1);
-  cp_async_commit();
-  const int g = lane >> 2, t4 = lane & 3;
-  const int b_row = (lane & 7) + (((lane >> 3) & 1) << 3);
-#pragma unroll 1
-  for (int kc = 0; kc < kNk; ++kc) {
-    if (kc + 2 < kNk) load(kc + 2, (kc + 2) % kOStages);
-    cp_async_commit();  // possibly empty: keeps one group per chunk
-    cp_async_wait<2>();  // chunk kc has landed
-    __syncthreads();
-    const uint8_t* a_p = smem_o + (kc % kOStages) * kOStageBytes;
-    const uint32_t b_s = sb + (kc % kOStages) * kOStageBytes + kOABytes;
-#pragma unroll
-    for (int ks = 0; ks < kOKc / 16; ++ks) {
-      // A fragment of m16n8k16 (rows g, g+8; k 2 t4, 2 t4 + 8), rounded to bf16 here.
-      uint32_t af[4];
-#pragma unroll
-      for (int hk = 0; hk < 2; ++hk) {
-        const int k = ks * 16 + 2 * t4 + 8 * hk;
-#pragma unroll
-        for (int hr = 0; hr < 2; ++hr) {
-          const int r = warp * 16 + g + 8 * hr;
-          const float2 v = *reinterpret_cast<const float2*>(a_p + r * 256 + (((k >> 2) ^ (r & 7)) * 16) + (k & 3) * 4);
-          af[hr + 2 * hk] = pack_bf16x2(v.x, v.y);
+    mbar_init(bar(kQDone), 1);
+    fence_mbar_init();
+    tma_prefetch_desc(&map_a);
+    tma_prefetch_desc(&map_b);
+    tma_prefetch_desc(&map_o);
+  }
+  if (warp == 5) {
+    tmem_alloc(smem_u32(&tmem_s), 256);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_s;
+  const Guard gd{err, &abort_s, limit_ns};
+
+  if (warp == 4) {
+    // ---------------------------------------------------------------- TMA loads
+    if (lane == 0) {
+      int it = 0, g = 0, ga = 0, gb = 0;  // items, n-tiles; loads issued into A and B
+      bool ok = true;
+      for (int item = blockIdx.x; ok && item < items; item += gridDim.x, ++it) {
+        const int h = item % H, b0 = (item / H) * kRows;
+        if (!wait_on(bar(kQAEmpty), (it & 1) ^ 1, gd)) { ok = false; break; }
+        mbar_expect_tx(bar(kQAFull), kQA);
+        tma_load_3d(sbase + kQSmA, &map_a, 0, h, b0, bar(kQAFull));
+        tma_load_3d(sbase + kQSmA + kBox, &map_a, 64, h, b0, bar(kQAFull));
+        ++ga;
+        for (int j = 0; j < kQNt; ++j, ++g) {
+          const int s = g % kQBStages;
+          if (!wait_on(bar(kQBEmpty + s), ((g / kQBStages) & 1) ^ 1, gd)) { ok = false; break; }
+          mbar_expect_tx(bar(kQBFull + s), kQB);
+          tma_load_3d(sbase + kQSmB + s * kQB, &map_b, 128 * j, 0, h, bar(kQBFull + s));
+          tma_load_3d(sbase + kQSmB + s * kQB + kBox, &map_b, 128 * j + 64, 0, h, bar(kQBFull + s));
+          ++gb;
         }
       }
-#pragma unroll
-      for (int nn = 0; nn < kTileN / 16; ++nn) {
-        uint32_t bf[4];
-        ldmatrix_x4_trans(bf, b_s + swz16(ks * 16 + b_row, nn * 2 + (lane >> 4)));
-        mma_bf16_16816(acc[2 * nn], af, bf[0], bf[1]);
-        mma_bf16_16816(acc[2 * nn + 1], af, bf[2], bf[3]);
+      // Every load issued lands before the CTA may exit (bounded).
+      if (ga > 0) drain_on(bar(kQAFull), (ga - 1) & 1, limit_ns);
+      for (int k = 0; k < kQBStages && k < gb; ++k) {
+        const int l = gb - 1 - k;
+        drain_on(bar(kQBFull + l % kQBStages), (l / kQBStages) & 1, limit_ns);
       }
     }
-    __syncthreads();  // the stage is refilled by the next iteration's load
+    __syncwarp();
+  } else if (warp == 5) {
+    // ---------------------------------------------------------------- MMA issue
+    if (lane == 0) {
+      int it = 0, g = 0;
+      bool ok = true;
+      for (int item = blockIdx.x; ok && item < items; item += gridDim.x, ++it) {
+        if (!wait_on(bar(kQAFull), it & 1, gd)) { ok = false; break; }
+        for (int j = 0; j < kQNt; ++j, ++g) {
+          const int s = g % kQBStages, d = g & 1;
+          if (!wait_on(bar(kQBFull + s), (g / kQBStages) & 1, gd) ||
+              !wait_on(bar(kQDEmpty + d), ((g >> 1) & 1) ^ 1, gd)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t ab = sbase + kQSmA, bb = sbase + kQSmB + s * kQB;
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            mma_ss(tmem + d * 128, desc_sw128(ab + (kk >> 2) * kBox + (kk & 3) * 32, 16, 1024),
+                   desc_sw128(bb + kk * 2048, kBox, 1024), kQIdesc, kk > 0 ? 1u : 0u);
+          mma_commit(bar(kQBEmpty + s));
+          mma_commit(bar(kQDFull + d));
+        }
+        if (!ok) break;
+        mma_commit(bar(kQAEmpty));
+      }
+      mma_commit(bar(kQDone));
+      drain_on(bar(kQDone), 0, limit_ns);
+    }
+    __syncwarp();
+  } else {
+    // ---------------------------------------------------------------- epilogue: thread = batch row
+    // The four warps meet at named barriers, so none of them leaves the loops early:
+    // after a failed wait they keep the same barrier sequence and skip the work.
+    const int r = 32 * warp + lane;
+    const uint32_t t_row = tmem + ((uint32_t)(32 * warp) << 16);
+    int it = 0, g = 0;
+    bool ok = true;
+    for (int item = blockIdx.x; item < items; item += gridDim.x, ++it) {
+      const int h = item % H, b0 = (item / H) * kRows;
+      const int b = b0 + r;
+      if (ok && b < B) {  // the rope half of q' is a copy
+        const uint4* src = reinterpret_cast<const uint4*>(q_rope + ((size_t)b * H + h) * kDRope);
+        uint4* dst = reinterpret_cast<uint4*>(q_out + ((size_t)b * H + h) * kDQK + kDLatent);
+#pragma unroll
+        for (int c = 0; c < 8; ++c) dst[c] = src[c];
+      }
+      for (int j = 0; j < kQNt; ++j, ++g) {
+        const int d = g & 1;
+        if (ok) ok = __all_sync(0xffffffffu, wait_on(bar(kQDFull + d), (g >> 1) & 1, gd));
+        tc_fence_after();
+        // Output buffer d was last stored from two n-tiles ago: that store has read it.
+        if (tid == 0) bulk_wait_read_1();
+        bar_sync_epilogue();
+        if (ok) {
+          uint8_t* ob = smem + kQSmO + d * kQO;
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {  // 32 columns at a time
+            uint32_t v[32];
+            tmem_ld32(t_row + d * 128 + 32 * c, v);
+            tmem_wait_ld();
+            uint8_t* row = ob + (c >> 1) * kBox + r * 128;
+#pragma unroll
+            for (int q4 = 0; q4 < 4; ++q4) {
+              const int chunk = (c & 1) * 4 + q4;
+              *reinterpret_cast<uint4*>(row + ((chunk ^ (r & 7)) * 16)) = pack8(v + 8 * q4);
+            }
+          }
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bar(kQDEmpty + d));
+          fence_proxy_async();
+        }
+        // Every epilogue warp agrees on ok here: a warp that failed set the abort flag,
+        // and the store below is issued only if all four wrote their rows.
+        bar_sync_epilogue();
+        if (tid == 0 && !abort_s) {
+          tma_store_3d(&map_o, sbase + kQSmO + d * kQO, 128 * j, h, b0);
+          tma_store_3d(&map_o, sbase + kQSmO + d * kQO + kBox, 128 * j + 64, h, b0);
+          bulk_commit();
+        }
+      }
+    }
+    if (tid == 0) bulk_wait_all();  // every store has completed before the CTA exits
   }
 
-#pragma unroll
-  for (int r = 0; r < 2; ++r) {
-    const int row = warp * 16 + g + r * 8;
-    if (row < rows) {
-      float* dst = out + ((size_t)(b0 + row) * H + h) * MLA_D_V + t4 * 2;
-#pragma unroll
-      for (int i = 0; i < 16; ++i) *reinterpret_cast<float2*>(dst + i * 8) = make_float2(acc[i][2 * r], acc[i][2 * r + 1]);
-    }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 5) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 256);
   }
+}
+
+// ================================================================ absorb_o
+// Item (head h, batch tile mt): K = 512 in eight chunks of 64.  Per chunk, TMA brings
+// the fp32 out_latent rows [128 x 64] (two 128B-swizzled boxes of 32 floats) and the
+// weights W_UV[h][64 k x 128 n] (two MN-major boxes); four converter warps round the
+// fp32 rows to bf16 (nearest even) into the K-major A operand; the MMA warp adds the
+// chunk's four K = 16 steps into D = 128 x 128 fp32 in TMEM.  The epilogue writes D
+// through shared memory by TMA stores.  Warps 0-3 epilogue, 4-7 convert, 8 TMA, 9 MMA.
+constexpr int kOThreads = 320;
+constexpr int kOF = 2 * kBox, kOA = kBox, kOB = kBox, kOO = 4 * kBox;  // 32, 16, 16, 64 KB
+constexpr int kOFStages = 2, kOStages = 3;
+constexpr int kOSmF = 0, kOSmA = kOFStages * kOF, kOSmB = kOSmA + kOStages * kOA, kOSmO = kOSmB + kOStages * kOB;
+constexpr int kOSmem = kOSmO + kOO;  // 224 KB
+constexpr int kOChunks = kDLatent / 64;
+constexpr uint32_t kOIdesc = idesc_bf16_f32(128, 128, 0, 1);
+
+enum OBar {
+  kOFFull = 0,
+  kOFEmpty = kOFFull + kOFStages,
+  kOBFull = kOFEmpty + kOFStages,
+  kOABEmpty = kOBFull + kOStages,  // MMA done with A and B of a stage
+  kOAReady = kOABEmpty + kOStages,
+  kODFull = kOAReady + kOStages,
+  kODEmpty = kODFull + 2,
+  kODone = kODEmpty + 2,
+  kONumBars
+};
+
+__global__ void __launch_bounds__(kOThreads, 1)
+    absorb_o_tc_kernel(const __grid_constant__ CUtensorMap map_f, const __grid_constant__ CUtensorMap map_w,
+                       const __grid_constant__ CUtensorMap map_o, int B, int H, int* err, uint64_t limit_ns) {
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ __align__(8) uint64_t bars[kONumBars];
+  __shared__ uint32_t tmem_s;
+  __shared__ int abort_s;
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  auto bar = [&](int i) { return smem_u32(&bars[i]); };
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int items = H * ((B + kRows - 1) / kRows);
+
+  if (tid == 0) {
+    abort_s = 0;
+    for (int i = 0; i < kOFStages; ++i) {
+      mbar_init(bar(kOFFull + i), 1);
+      mbar_init(bar(kOFEmpty + i), 4);  // one arrival per converter warp
+    }
+    for (int i = 0; i < kOStages; ++i) {
+      mbar_init(bar(kOBFull + i), 1);
+      mbar_init(bar(kOABEmpty + i), 1);
+      mbar_init(bar(kOAReady + i), 4);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(bar(kODFull + i), 1);
+      mbar_init(bar(kODEmpty + i), 4);
+    }
+    mbar_init(bar(kODone), 1);
+    fence_mbar_init();
+    tma_prefetch_desc(&map_f);
+    tma_prefetch_desc(&map_w);
+    tma_prefetch_desc(&map_o);
+  }
+  if (warp == 9) {
+    tmem_alloc(smem_u32(&tmem_s), 256);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_s;
+  const Guard gd{err, &abort_s, limit_ns};
+
+  if (warp == 8) {
+    // ---------------------------------------------------------------- TMA loads
+    if (lane == 0) {
+      int gf = 0, gb = 0;  // fp32 A and weight chunks issued
+      bool ok = true;
+      for (int item = blockIdx.x; ok && item < items; item += gridDim.x) {
+        const int h = item % H, b0 = (item / H) * kRows;
+        for (int c = 0; c < kOChunks; ++c) {
+          const int f = gf % kOFStages, s = gb % kOStages;
+          if (!wait_on(bar(kOFEmpty + f), ((gf / kOFStages) & 1) ^ 1, gd)) { ok = false; break; }
+          mbar_expect_tx(bar(kOFFull + f), kOF);
+          tma_load_3d(sbase + kOSmF + f * kOF, &map_f, 64 * c, h, b0, bar(kOFFull + f));
+          tma_load_3d(sbase + kOSmF + f * kOF + kBox, &map_f, 64 * c + 32, h, b0, bar(kOFFull + f));
+          ++gf;
+          if (!wait_on(bar(kOABEmpty + s), ((gb / kOStages) & 1) ^ 1, gd)) { ok = false; break; }
+          mbar_expect_tx(bar(kOBFull + s), kOB);
+          tma_load_3d(sbase + kOSmB + s * kOB, &map_w, 0, 64 * c, h, bar(kOBFull + s));
+          tma_load_3d(sbase + kOSmB + s * kOB + kBox / 2, &map_w, 64, 64 * c, h, bar(kOBFull + s));
+          ++gb;
+        }
+      }
+      // Every load issued lands before the CTA may exit (bounded).
+      for (int k = 0; k < kOFStages && k < gf; ++k) {
+        const int l = gf - 1 - k;
+        drain_on(bar(kOFFull + l % kOFStages), (l / kOFStages) & 1, limit_ns);
+      }
+      for (int k = 0; k < kOStages && k < gb; ++k) {
+        const int l = gb - 1 - k;
+        drain_on(bar(kOBFull + l % kOStages), (l / kOStages) & 1, limit_ns);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 9) {
+    // ---------------------------------------------------------------- MMA issue
+    if (lane == 0) {
+      int it = 0, g = 0;
+      bool ok = true;
+      for (int item = blockIdx.x; ok && item < items; item += gridDim.x, ++it) {
+        const int d = it & 1;
+        if (!wait_on(bar(kODEmpty + d), ((it >> 1) & 1) ^ 1, gd)) { ok = false; break; }
+        for (int c = 0; c < kOChunks; ++c, ++g) {
+          const int s = g % kOStages;
+          if (!wait_on(bar(kOAReady + s), (g / kOStages) & 1, gd) || !wait_on(bar(kOBFull + s), (g / kOStages) & 1, gd)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t ab = sbase + kOSmA + s * kOA, bb = sbase + kOSmB + s * kOB;
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            mma_ss(tmem + d * 128, desc_sw128(ab + kk * 32, 16, 1024), desc_sw128(bb + kk * 2048, kBox / 2, 1024),
+                   kOIdesc, (c > 0 || kk > 0) ? 1u : 0u);
+          mma_commit(bar(kOABEmpty + s));
+        }
+        if (!ok) break;
+        mma_commit(bar(kODFull + d));
+      }
+      mma_commit(bar(kODone));
+      drain_on(bar(kODone), 0, limit_ns);
+    }
+    __syncwarp();
+  } else if (warp >= 4) {
+    // ---------------------------------------------------------------- fp32 -> bf16 A: thread = batch row
+    const int r = tid - 128;
+    int g = 0;
+    bool ok = true;
+    for (int item = blockIdx.x; ok && item < items; item += gridDim.x) {
+      for (int c = 0; c < kOChunks; ++c, ++g) {
+        const int f = g % kOFStages, s = g % kOStages;
+        if (!__all_sync(0xffffffffu, wait_on(bar(kOFFull + f), (g / kOFStages) & 1, gd) &&
+                                         wait_on(bar(kOABEmpty + s), ((g / kOStages) & 1) ^ 1, gd))) {
+          ok = false;
+          break;
+        }
+        const uint8_t* frow = smem + kOSmF + f * kOF + r * 128;
+        uint8_t* arow = smem + kOSmA + s * kOA + r * 128;
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {  // bf16 chunk q: k 8q..8q+7 = fp32 box q/4, chunks 2(q%4), 2(q%4)+1
+          const uint8_t* fb = frow + (q >> 2) * kBox;
+          const int c0 = 2 * (q & 3);
+          const float4 x = *reinterpret_cast<const float4*>(fb + ((c0 ^ (r & 7)) * 16));
+          const float4 y = *reinterpret_cast<const float4*>(fb + (((c0 + 1) ^ (r & 7)) * 16));
+          *reinterpret_cast<uint4*>(arow + ((q ^ (r & 7)) * 16)) =
+              make_uint4(pack_bf16x2(x.x, x.y), pack_bf16x2(x.z, x.w), pack_bf16x2(y.x, y.y), pack_bf16x2(y.z, y.w));
+        }
+        fence_proxy_async();
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(bar(kOFEmpty + f));
+          mbar_arrive(bar(kOAReady + s));
+        }
+      }
+    }
+  } else {
+    // ---------------------------------------------------------------- epilogue: thread = batch row
+    // As in absorb_q, the four warps keep the same named-barrier sequence after a failure.
+    const int r = 32 * warp + lane;
+    const uint32_t t_row = tmem + ((uint32_t)(32 * warp) << 16);
+    int it = 0;
+    bool ok = true;
+    for (int item = blockIdx.x; item < items; item += gridDim.x, ++it) {
+      const int h = item % H, b0 = (item / H) * kRows;
+      const int d = it & 1;
+      if (ok) ok = __all_sync(0xffffffffu, wait_on(bar(kODFull + d), (it >> 1) & 1, gd));
+      tc_fence_after();
+      if (tid == 0) bulk_wait_all();  // the previous item's store has finished with the buffer
+      bar_sync_epilogue();
+      if (ok) {
+        uint8_t* row = smem + kOSmO + r * 128;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {  // 32 columns = one box
+          uint32_t v[32];
+          tmem_ld32(t_row + d * 128 + 32 * c, v);
+          tmem_wait_ld();
+#pragma unroll
+          for (int q = 0; q < 8; ++q)
+            *reinterpret_cast<uint4*>(row + c * kBox + ((q ^ (r & 7)) * 16)) =
+                make_uint4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(kODEmpty + d));
+        fence_proxy_async();
+      }
+      bar_sync_epilogue();
+      if (tid == 0 && !abort_s) {
+#pragma unroll
+        for (int c = 0; c < 4; ++c) tma_store_3d(&map_o, sbase + kOSmO + c * kBox, 32 * c, h, b0);
+        bulk_commit();
+      }
+    }
+    if (tid == 0) bulk_wait_all();
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 9) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 256);
+  }
+}
+
+// ---------------------------------------------------------------- host side
+PFN_cuTensorMapEncodeTiled_v12000 encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = [] {
+    cudaDriverEntryPointQueryResult q;
+    void* p = nullptr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    return static_cast<PFN_cuTensorMapEncodeTiled_v12000>(nullptr);
+  }();
+  return fn;
+}
+
+// 3-D tiled map: dims innermost first (elements), strides of dims 1 and 2 in bytes.
+bool map3d(CUtensorMap* m, CUtensorMapDataType t, const void* base, uint64_t d0, uint64_t d1, uint64_t d2,
+           uint64_t s1, uint64_t s2, uint32_t b0, uint32_t b1, uint32_t b2, CUtensorMapSwizzle sw) {
+  auto enc = encoder();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {d0, d1, d2};
+  cuuint64_t strides[2] = {s1, s2};
+  cuuint32_t box[3] = {b0, b1, b2};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return enc(m, t, 3, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int sm_count() {
+  static int n = 0;
+  if (n == 0) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (n <= 0) n = 1;
+  }
+  return n;
 }
 
 }  // namespace
 
 cudaError_t launch_absorb_q(const __nv_bfloat16* q_nope, const __nv_bfloat16* q_rope, const __nv_bfloat16* w_uk,
-                            __nv_bfloat16* q_out, int batch, int heads, cudaStream_t stream) {
-  dim3 grid((batch + kTileM - 1) / kTileM, kDLatent / kTileN, heads);
-  absorb_q_kernel<<<grid, kThreads, 0, stream>>>(q_nope, q_rope, w_uk, q_out, batch, heads);
+                            __nv_bfloat16* q_out, int batch, int heads, int* err, cudaStream_t stream) {
+  CUtensorMap ma, mb, mo;
+  const uint64_t H = heads, Bn = batch;
+  const auto bf = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  const auto sw = CU_TENSOR_MAP_SWIZZLE_128B;
+  if (!map3d(&ma, bf, q_nope, MLA_D_NOPE, H, Bn, MLA_D_NOPE * 2, H * MLA_D_NOPE * 2, 64, 1, kRows, sw) ||
+      !map3d(&mb, bf, w_uk, kDLatent, MLA_D_NOPE, H, kDLatent * 2, (uint64_t)MLA_D_NOPE * kDLatent * 2, 64,
+             MLA_D_NOPE, 1, sw) ||
+      !map3d(&mo, bf, q_out, kDQK, H, Bn, kDQK * 2, H * kDQK * 2, 64, 1, kRows, sw))
+    return cudaErrorInvalidValue;
+  const int smem = kQSmem + 1024;
+  cudaError_t e = cudaFuncSetAttribute(absorb_q_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  const int items = heads * ((batch + kRows - 1) / kRows);
+  const int grid = items < sm_count() ? items : sm_count();
+  absorb_q_tc_kernel<<<grid, kThreads, smem, stream>>>(ma, mb, mo, q_rope, q_out, batch, heads, err,
+                                                       2000ull * 1000000ull);
   return cudaGetLastError();
 }
 
 cudaError_t launch_absorb_o(const float* out_latent, const __nv_bfloat16* w_uv, float* out, int batch, int heads,
-                            cudaStream_t stream) {
-  // 96 KB of dynamic shared memory (set on every call: the attribute is per device).
-  const cudaError_t attr = cudaFuncSetAttribute(absorb_o_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kOSmem);
-  if (attr != cudaSuccess) return attr;
-  dim3 grid((batch + kTileM - 1) / kTileM, heads);
-  absorb_o_kernel<<<grid, kThreads, kOSmem, stream>>>(out_latent, w_uv, out, batch, heads);
+                            int* err, cudaStream_t stream) {
+  CUtensorMap mf, mw, mo;
+  const uint64_t H = heads, Bn = batch;
+  const auto sw = CU_TENSOR_MAP_SWIZZLE_128B;
+  if (!map3d(&mf, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, out_latent, kDLatent, H, Bn, kDLatent * 4, H * kDLatent * 4, 32, 1,
+             kRows, sw) ||
+      !map3d(&mw, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, w_uv, MLA_D_V, kDLatent, H, MLA_D_V * 2,
+             (uint64_t)kDLatent * MLA_D_V * 2, 64, 64, 1, sw) ||
+      !map3d(&mo, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, out, MLA_D_V, H, Bn, MLA_D_V * 4, H * MLA_D_V * 4, 32, 1, kRows, sw))
+    return cudaErrorInvalidValue;
+  const int smem = kOSmem + 1024;
+  cudaError_t e = cudaFuncSetAttribute(absorb_o_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  const int items = heads * ((batch + kRows - 1) / kRows);
+  const int grid = items < sm_count() ? items : sm_count();
+  absorb_o_tc_kernel<<<grid, kOThreads, smem, stream>>>(mf, mw, mo, batch, heads, err, 2000ull * 1000000ull);
   return cudaGetLastError();
 }
 

@@ -340,9 +340,13 @@ mla_status_t mla_absorb_q(const void* q_nope, const void* q_rope, const void* w_
   if (heads < 1 || heads > MLA_MAX_HEADS) return fail(MLA_ERR_UNSUPPORTED, "heads = %d outside [1, 128]", heads);
   if (!aligned16(q_nope) || !aligned16(q_rope) || !aligned16(w_uk) || !aligned16(q_out))
     return fail(MLA_ERR_INVALID_ARG, "absorb_q operands must be 16-byte aligned");
+  std::lock_guard<std::mutex> lk(g_mu);
+  DeviceState* d = nullptr;
+  mla_status_t s = device_state(&d);
+  if (s != MLA_OK) return s;
   cudaError_t e = launch_absorb_q(static_cast<const __nv_bfloat16*>(q_nope), static_cast<const __nv_bfloat16*>(q_rope),
                                   static_cast<const __nv_bfloat16*>(w_uk), static_cast<__nv_bfloat16*>(q_out), batch,
-                                  heads, reinterpret_cast<cudaStream_t>(stream));
+                                  heads, d->err, reinterpret_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? MLA_OK : cuda_fail(e, "absorb_q launch");
 }
 
@@ -354,7 +358,11 @@ mla_status_t mla_absorb_o(const float* out_latent, const void* w_uv, float* out,
   if (heads < 1 || heads > MLA_MAX_HEADS) return fail(MLA_ERR_UNSUPPORTED, "heads = %d outside [1, 128]", heads);
   if (!aligned16(out_latent) || !aligned16(w_uv) || !aligned16(out))
     return fail(MLA_ERR_INVALID_ARG, "absorb_o operands must be 16-byte aligned");
-  cudaError_t e = launch_absorb_o(out_latent, static_cast<const __nv_bfloat16*>(w_uv), out, batch, heads,
+  std::lock_guard<std::mutex> lk(g_mu);
+  DeviceState* d = nullptr;
+  mla_status_t s = device_state(&d);
+  if (s != MLA_OK) return s;
+  cudaError_t e = launch_absorb_o(out_latent, static_cast<const __nv_bfloat16*>(w_uv), out, batch, heads, d->err,
                                   reinterpret_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? MLA_OK : cuda_fail(e, "absorb_o launch");
 }

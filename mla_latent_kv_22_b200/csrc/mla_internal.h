@@ -70,10 +70,10 @@ cudaError_t launch_decode_mma(const DecodeArgs& a, cudaStream_t stream);
 int decode_mma_heads_per_cta();
 cudaError_t launch_combine(const DecodeArgs& a, cudaStream_t stream);
 cudaError_t launch_absorb_q(const __nv_bfloat16* q_nope, const __nv_bfloat16* q_rope,
-                            const __nv_bfloat16* w_uk, __nv_bfloat16* q_out, int batch, int heads,
+                            const __nv_bfloat16* w_uk, __nv_bfloat16* q_out, int batch, int heads, int* err,
                             cudaStream_t stream);
 cudaError_t launch_absorb_o(const float* out_latent, const __nv_bfloat16* w_uv, float* out, int batch,
-                            int heads, cudaStream_t stream);
+                            int heads, int* err, cudaStream_t stream);
 
 // Defined in api.cu: the per-device decode plan, the thread's last-error text,
 // and raw knob values.
