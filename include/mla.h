@@ -119,10 +119,12 @@ mla_status_t mla_decode(const void* q, const void* kv_cache, const int32_t* bloc
  * new tokens appended to the cache before the call.  Each query row is computed as
  * in mla_decode (s_q = 1 gives exactly mla_decode), with the s_q x heads rows of a
  * sequence sharing every load of its cached rows.
- * s_q >= 1 and s_q * heads <= 128, else MLA_ERR_UNSUPPORTED; it runs on the
- * tcgen05 kernel only (MLA_ERR_UNSUPPORTED if the kernel knob forces the other).
- * Every other argument, the workspace, determinism and error behaviour are those
- * of mla_decode (mla_workspace_size takes s_q * heads as its heads).
+ * s_q >= 1, heads <= 128 and s_q * heads <= 2048, else MLA_ERR_UNSUPPORTED.
+ * Up to 128 rows share one pass over the cache; more rows run as groups of 128,
+ * each group reading the cache again.  It runs on the tcgen05 kernel only
+ * (MLA_ERR_UNSUPPORTED if the kernel knob forces the other).  Every other
+ * argument, the workspace, determinism and error behaviour are those of
+ * mla_decode (mla_workspace_size takes s_q * heads as its heads).
  */
 mla_status_t mla_decode_multi(const void* q, const void* kv_cache, const int32_t* block_table,
                               const int32_t* cache_seqlens, float* out, float* lse,

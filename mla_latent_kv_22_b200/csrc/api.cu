@@ -194,9 +194,10 @@ size_t mla_workspace_size(int batch, int heads, int max_blocks) {
   std::lock_guard<std::mutex> lk(g_mu);
   DeviceState* d = nullptr;
   if (device_state(&d) != MLA_OK) return 0;
-  const int kernel = pick_kernel(heads);
-  const int P = num_workers_for(*d, kernel < 0 ? 1 : kernel, heads);
-  return carve_schedule(nullptr, batch, heads, P, nullptr);
+  const int group = std::min(heads, (int)MLA_MAX_HEADS);  // rows per decode launch
+  const int kernel = pick_kernel(group);
+  const int P = num_workers_for(*d, kernel < 0 ? 1 : kernel, group);
+  return carve_schedule(nullptr, batch, group, P, nullptr);
 }
 
 mla_status_t mla_set_workspace(void* dev_ptr, size_t bytes) {
@@ -241,7 +242,11 @@ namespace mla {
 namespace {
 
 // mla_decode and mla_decode_multi: `heads` rows per sequence, made of s_q query
-// tokens of heads / s_q heads each.
+// tokens of heads / s_q heads each.  More than 128 rows (s_q > 1 only) run as groups of
+// at most 128 rows, each a decode and a combine over the same schedule: every group
+// reads the cache once more.
+constexpr int kMaxRows = 16 * MLA_MAX_HEADS;  // query rows per sequence for mla_decode_multi
+
 mla_status_t decode_call(const void* q, const void* kv_cache, const int32_t* block_table, const int32_t* cache_seqlens,
                          float* out, float* lse, int batch, int s_q, int heads, int num_pages, int max_blocks,
                          float softmax_scale, mla_stream_t stream_) {
@@ -252,7 +257,8 @@ mla_status_t decode_call(const void* q, const void* kv_cache, const int32_t* blo
   if (batch == 0) return MLA_OK;
   if (!q || !kv_cache || !cache_seqlens || !out || !lse)
     return fail(MLA_ERR_INVALID_ARG, "null pointer argument");
-  if (heads < 1 || heads > MLA_MAX_HEADS) return fail(MLA_ERR_UNSUPPORTED, "heads = %d outside [1, 128]", heads);
+  if (heads < 1 || heads > (s_q > 1 ? kMaxRows : MLA_MAX_HEADS))
+    return fail(MLA_ERR_UNSUPPORTED, "%d rows per sequence outside [1, %d]", heads, s_q > 1 ? kMaxRows : MLA_MAX_HEADS);
   if (max_blocks < 1) return fail(MLA_ERR_INVALID_ARG, "max_blocks must be >= 1");
   if (block_table && num_pages < 1) return fail(MLA_ERR_INVALID_ARG, "paged cache with num_pages < 1");
   if ((long long)batch * max_blocks > (1LL << 31) - 1 || (long long)max_blocks * MLA_PAGE_TOKENS > (1LL << 30))
@@ -268,11 +274,12 @@ mla_status_t decode_call(const void* q, const void* kv_cache, const int32_t* blo
   DeviceState* d = nullptr;
   mla_status_t s = device_state(&d);
   if (s != MLA_OK) return s;
-  const int kernel = pick_kernel(heads);
+  const int group = std::min(heads, (int)MLA_MAX_HEADS);  // rows per launch
+  const int kernel = pick_kernel(group);
   if (kernel < 0) return fail(MLA_ERR_UNSUPPORTED, "requested decode kernel does not handle heads = %d", heads);
   if (s_q > 1 && kernel != 2) return fail(MLA_ERR_UNSUPPORTED, "several query tokens need the tcgen05 kernel");
-  const int P = num_workers_for(*d, kernel, heads);
-  const size_t need = carve_schedule(nullptr, batch, heads, P, nullptr);
+  const int P = num_workers_for(*d, kernel, group);
+  const size_t need = carve_schedule(nullptr, batch, group, P, nullptr);
   s = ensure_workspace(*d, need, stream);
   if (s != MLA_OK) return s;
 
@@ -284,27 +291,33 @@ mla_status_t decode_call(const void* q, const void* kv_cache, const int32_t* blo
   a.out = out;
   a.lse = lse;
   a.batch = batch;
-  a.heads = heads;
+  a.heads = group;
   a.num_pages = num_pages;
   a.max_blocks = max_blocks;
   a.scale = softmax_scale;
   a.err = d->err;
-  carve_schedule(d->ws, batch, heads, P, &a.sched);
+  carve_schedule(d->ws, batch, group, P, &a.sched);
   a.wait_limit = g_knobs[MLA_KNOB_WAIT_LIMIT].load() > 0 ? g_knobs[MLA_KNOB_WAIT_LIMIT].load() : 2000;  // ms
   a.withhold_arrive = g_knobs[MLA_KNOB_WITHHOLD_ARRIVE].load();
   a.s_q = s_q;
   a.hq = heads / s_q;
+  a.row_stride = heads;
+  a.row0 = 0;
   const int min_pages = g_knobs[MLA_KNOB_MIN_PAGES].load() > 0 ? g_knobs[MLA_KNOB_MIN_PAGES].load() : 4;
 
   record_event(*d, 0, stream);
   cudaError_t e = launch_schedule(cache_seqlens, batch, max_blocks, min_pages, a.sched, d->err, stream);
   if (e != cudaSuccess) return cuda_fail(e, "schedule launch");
   record_event(*d, 1, stream);
-  e = kernel == 2 ? launch_decode_tc(a, stream) : launch_decode_mma(a, stream);
-  if (e != cudaSuccess) return cuda_fail(e, "decode launch");
-  record_event(*d, 2, stream);
-  e = launch_combine(a, stream);
-  if (e != cudaSuccess) return cuda_fail(e, "combine launch");
+  for (int r0 = 0; r0 < heads; r0 += group) {
+    a.row0 = r0;
+    a.heads = std::min(group, heads - r0);
+    e = kernel == 2 ? launch_decode_tc(a, stream) : launch_decode_mma(a, stream);
+    if (e != cudaSuccess) return cuda_fail(e, "decode launch");
+    if (r0 + group >= heads) record_event(*d, 2, stream);
+    e = launch_combine(a, stream);
+    if (e != cudaSuccess) return cuda_fail(e, "combine launch");
+  }
   record_event(*d, 3, stream);
   if (g_timing.load()) d->timed_calls++;
   return MLA_OK;
@@ -326,8 +339,9 @@ mla_status_t mla_decode_multi(const void* q, const void* kv_cache, const int32_t
                               const int32_t* cache_seqlens, float* out, float* lse, int batch, int s_q, int heads,
                               int num_pages, int max_blocks, float softmax_scale, mla_stream_t stream) {
   if (s_q < 1 || heads < 0) return fail(MLA_ERR_INVALID_ARG, "s_q = %d, heads = %d", s_q, heads);
-  if ((long long)s_q * heads > MLA_MAX_HEADS)
-    return fail(MLA_ERR_UNSUPPORTED, "s_q x heads = %lld rows > 128", (long long)s_q * heads);
+  if (heads > MLA_MAX_HEADS) return fail(MLA_ERR_UNSUPPORTED, "heads = %d > 128", heads);
+  if ((long long)s_q * heads > kMaxRows)
+    return fail(MLA_ERR_UNSUPPORTED, "s_q x heads = %lld rows > %d", (long long)s_q * heads, kMaxRows);
   return decode_call(q, kv_cache, block_table, cache_seqlens, out, lse, batch, s_q, s_q * heads, num_pages,
                      max_blocks, softmax_scale, stream);
 }

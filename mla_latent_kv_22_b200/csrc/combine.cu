@@ -25,13 +25,14 @@ __global__ void __launch_bounds__(kWarps * 32) combine_kernel(DecodeArgs a) {
   if (h >= a.heads) return;
   const Schedule& sc = a.sched;
   const SeqInfo si = sc.seq[b];
-  float4* out4 = reinterpret_cast<float4*>(a.out + ((size_t)b * a.heads + h) * kDLatent);
+  const size_t orow = (size_t)b * a.row_stride + a.row0 + h;  // this row in out and lse
+  float4* out4 = reinterpret_cast<float4*>(a.out + orow * kDLatent);
   if (si.num_pieces == 1) return;
   if (si.num_pieces <= 0) {
     const float v = si.num_pieces == 0 ? 0.f : NAN;
 #pragma unroll
     for (int i = 0; i < 4; ++i) out4[lane + 32 * i] = make_float4(v, v, v, v);
-    if (lane == 0) a.lse[(size_t)b * a.heads + h] = si.num_pieces == 0 ? -INFINITY : NAN;
+    if (lane == 0) a.lse[orow] = si.num_pieces == 0 ? -INFINITY : NAN;
     return;
   }
   const int np = si.num_pieces;
@@ -70,7 +71,7 @@ __global__ void __launch_bounds__(kWarps * 32) combine_kernel(DecodeArgs a) {
     const float v = nan ? NAN : 0.f;
 #pragma unroll
     for (int i = 0; i < 4; ++i) out4[lane + 32 * i] = make_float4(v, v, v, v);
-    if (lane == 0) a.lse[(size_t)b * a.heads + h] = nan ? NAN : -INFINITY;
+    if (lane == 0) a.lse[orow] = nan ? NAN : -INFINITY;
     return;
   }
 
@@ -102,7 +103,7 @@ __global__ void __launch_bounds__(kWarps * 32) combine_kernel(DecodeArgs a) {
 #pragma unroll
   for (int i = 0; i < 4; ++i)
     out4[lane + 32 * i] = make_float4(acc[i].x * inv, acc[i].y * inv, acc[i].z * inv, acc[i].w * inv);
-  if (lane == 0) a.lse[(size_t)b * a.heads + h] = L + logf(wsum);
+  if (lane == 0) a.lse[orow] = L + logf(wsum);
 }
 
 }  // namespace

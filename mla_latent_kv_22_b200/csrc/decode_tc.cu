@@ -544,13 +544,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       const int b = pc.b, n = pc.pe - pc.pa;
       const int T = a.seqlens[b];
       // Tokens this row attends to: all T, or its query token's causal window.
-      const int Tq = kCausal && row < a.heads ? T - (a.s_q - 1 - row / a.hq) : T;
+      const int Tq = kCausal && row < a.heads ? T - (a.s_q - 1 - (a.row0 + row) / a.hq) : T;
       // ---- stage q' for this sequence into TMEM: this CTA's latent half (split
       // between the two warps of each lane quadrant) and its 32 rope dims
       {
         uint32_t qv[16];
         const bool live = qrow < a.heads;
-        const uint4* src = reinterpret_cast<const uint4*>(a.q + ((size_t)b * a.heads + (live ? qrow : 0)) * kDQK);
+        const size_t qbase = kCausal ? (size_t)b * a.row_stride + a.row0 : (size_t)b * a.heads;
+        const uint4* src = reinterpret_cast<const uint4*>(a.q + (qbase + (live ? qrow : 0)) * kDQK);
 #pragma unroll
         for (int c = 0; c < 4; ++c) {  // 4 x 32 dims of this warp's 128 latent dims
 #pragma unroll
@@ -721,8 +722,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       float* obase;
       float* lbase;
       if (complete) {
-        obase = a.out + (size_t)b * a.heads * kDLatent;
-        lbase = a.lse + (size_t)b * a.heads;
+        const size_t rbase = kCausal ? (size_t)b * a.row_stride + a.row0 : (size_t)b * a.heads;
+        obase = a.out + rbase * kDLatent;
+        lbase = a.lse + rbase;
       } else {
         const int slot = (b == sc.ranges[w].b0) ? w : P + w;
         obase = sc.part_o + (size_t)slot * a.heads * kDLatent;

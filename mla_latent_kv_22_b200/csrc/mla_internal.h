@@ -58,10 +58,11 @@ struct DecodeArgs {
   Schedule sched;
   int wait_limit;       // bounded-wait time limit in milliseconds (tcgen05 kernel)
   int withhold_arrive;  // test hook (tcgen05 kernel)
-  // Several query tokens per sequence (tcgen05 kernel only): the `heads` rows of a
-  // sequence are s_q query tokens of hq heads each (row r = query r / hq), and query
-  // i sees the first T - s_q + 1 + i cached tokens.  s_q = 1, hq = heads otherwise.
-  int s_q, hq;
+  // Several query tokens per sequence (tcgen05 kernel only): a sequence has
+  // row_stride = s_q x hq query rows in q, out and lse (row r = query r / hq; query i
+  // sees the first T - s_q + 1 + i cached tokens), of which one launch handles the
+  // `heads` rows starting at row0.  s_q = 1, hq = row_stride = heads, row0 = 0 otherwise.
+  int s_q, hq, row_stride, row0;
 };
 
 cudaError_t launch_schedule(const int32_t* seqlens, int batch, int max_blocks, int min_pages,

@@ -117,6 +117,8 @@ extern "C" mla_status_t mla_decode_noalloc(const void* q, const void* kv_cache, 
   a.withhold_arrive = 0;
   a.s_q = 1;
   a.hq = heads;
+  a.row_stride = heads;
+  a.row0 = 0;
   const int mp = mla::knob_value(MLA_KNOB_MIN_PAGES);
   const int min_pages = mp > 0 ? mp : 4;
 

@@ -57,8 +57,8 @@ def test_decode_host_validation(kw, status):
 
 
 @pytest.mark.parametrize("s_q,H,q,status", [
-    (0, 64, 16, 1), (-1, 64, 16, 1), (2, -1, 16, 1), (2, 65, 16, 2), (3, 43, 16, 2), (2, 64, None, 1), (2, 64, 24, 1),
-    (1, 129, 16, 2),
+    (0, 64, 16, 1), (-1, 64, 16, 1), (2, -1, 16, 1), (2, 129, 16, 2), (17, 128, 16, 2), (2049, 1, 16, 2),
+    (2, 64, None, 1), (2, 64, 24, 1), (1, 129, 16, 2),
 ])
 def test_decode_multi_host_validation(s_q, H, q, status):
     assert M.lib.mla_decode_multi(q, 16, None, 16, 16, 16, 2, s_q, H, 10, 4, 0.1, None) == status

@@ -5,8 +5,8 @@ Same tolerances as the single-token decode: |out - ref| <= 1e-2 + 1e-2 |ref|
 elementwise, |lse - ref| <= 2e-3, and rows whose window is empty must be exactly
 out = 0, lse = -inf.  The cases cover windows that are empty for some queries
 (T < s_q), windows that end inside the previous page, split sequences whose last
-piece holds no token of some queries' windows, 8 x 16 = 128 rows, and row counts
-that are not a multiple of 16.
+piece holds no token of some queries' windows, 8 x 16 = 128 rows, row counts
+that are not a multiple of 16, and more than 128 rows (run as groups of 128).
 """
 import numpy as np
 import pytest
@@ -51,6 +51,8 @@ def _ref(c, q_np):
     (4, 8, 16, [0, 7, 64, 513]),     # 128 rows; an empty sequence; a window ending at a page end
     (2, 3, 40, [130, 2]),            # 120 rows
     (5, 2, 1, [65, 64, 63, 1, 2]),   # one head per query token
+    (2, 2, 128, [300, 5]),           # 256 rows: two groups of 128
+    (3, 3, 50, [1, 100, 129]),       # 150 rows: groups of 128 and 22
 ])
 def test_multi_matches_oracle(B, s_q, H, lens):
     c, q = _case(B, s_q, H, lens, seed=70 + s_q * H, poison=True)
@@ -63,16 +65,18 @@ def test_multi_matches_oracle(B, s_q, H, lens):
 
 
 @pytest.mark.parametrize("workers", [1, 5, 40])
-def test_multi_split_pieces_without_tokens_for_some_queries(workers):
+@pytest.mark.parametrize("H", [32, 96])
+def test_multi_split_pieces_without_tokens_for_some_queries(workers, H):
     # 65 pages with one token on the last: at 2 pages per worker the last worker's
     # piece holds token 4096 only, which queries 0..2 of s_q = 4 do not see, so their
-    # partial for that piece is empty and the combine must give it zero weight.
+    # partial for that piece is empty and the combine must give it zero weight.  At
+    # H = 96 the 384 rows run as three groups over the same schedule.
     M.mla_set_knob("min_pages", 1)
     M.mla_set_knob("num_workers", workers)
-    c, q = _case(2, 4, 32, [4097, 300], seed=81, poison=True)
-    out, lse, err = _run(c, q, 4, 32)
+    c, q = _case(2, 4, H, [4097, 300], seed=81, poison=True)
+    out, lse, err = _run(c, q, 4, H)
     assert err == 0
-    assert_close(out, lse, *_ref(c, q), f"{workers} workers")
+    assert_close(out, lse, *_ref(c, q), f"{workers} workers, H={H}")
 
 
 def test_multi_single_token_is_bit_exact_decode():
@@ -99,9 +103,9 @@ def test_multi_paged_equals_contiguous_bit_exact():
 def test_multi_rejects_what_it_does_not_handle():
     c, q = _case(2, 2, 64, [100, 5], seed=84, poison=False)
     dev = upload(c)
-    too_many = torch.zeros(2, 3, 64, 576, dtype=torch.bfloat16, device="cuda")  # 192 rows
-    out = torch.zeros(2, 3, 64, 512, device="cuda")
-    lse = torch.zeros(2, 3, 64, device="cuda")
+    too_many = torch.zeros(2, 17, 128, 576, dtype=torch.bfloat16, device="cuda")  # 2176 rows
+    out = torch.zeros(2, 17, 128, 512, device="cuda")
+    lse = torch.zeros(2, 17, 128, device="cuda")
     with pytest.raises(M.MlaError) as ei:
         M.mla_decode_multi(too_many, dev[1], dev[2], dev[3], out, lse, c.softmax_scale)
     assert ei.value.name == "MLA_ERR_UNSUPPORTED"
