@@ -149,6 +149,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  // Launched as a programmatic dependent: the set-up above overlaps the previous grid,
+  // whose writes (the inputs) are complete and visible after this wait.
+  if (tid == 0) grid_dep_launch_dependents();
+  grid_dep_wait();
   const uint32_t tmem = tmem_s;
   const Guard gd{err, &abort_s, limit_ns};
 
@@ -343,6 +347,8 @@ __global__ void __launch_bounds__(kOThreads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  if (tid == 0) grid_dep_launch_dependents();
+  grid_dep_wait();  // as in absorb_q: the inputs are complete from here on
   const uint32_t tmem = tmem_s;
   const Guard gd{err, &abort_s, limit_ns};
 
@@ -526,6 +532,23 @@ cudaError_t allow_smem(const void* kernel, int bytes, bool (&done)[64]) {
   return e;
 }
 
+// Launch as a programmatic dependent of the previous grid on the stream.
+template <typename... Params, typename... Args>
+cudaError_t launch_dependent(void (*kernel)(Params...), int grid, int threads, int smem, cudaStream_t stream,
+                             Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid, 1, 1);
+  cfg.blockDim = dim3(threads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
 int sm_count() {
   static int n = 0;
   if (n == 0) {
@@ -556,9 +579,8 @@ cudaError_t launch_absorb_q(const __nv_bfloat16* q_nope, const __nv_bfloat16* q_
   if (e != cudaSuccess) return e;
   const int items = heads * ((batch + kRows - 1) / kRows);
   const int grid = items < sm_count() ? items : sm_count();
-  absorb_q_tc_kernel<<<grid, kThreads, smem, stream>>>(ma, mb, mo, q_rope, q_out, batch, heads, err,
-                                                       2000ull * 1000000ull);
-  return cudaGetLastError();
+  return launch_dependent(absorb_q_tc_kernel, grid, kThreads, smem, stream, ma, mb, mo, q_rope, q_out, batch, heads,
+                          err, 2000ull * 1000000ull);
 }
 
 cudaError_t launch_absorb_o(const float* out_latent, const __nv_bfloat16* w_uv, float* out, int batch, int heads,
@@ -578,8 +600,8 @@ cudaError_t launch_absorb_o(const float* out_latent, const __nv_bfloat16* w_uv, 
   if (e != cudaSuccess) return e;
   const int items = heads * ((batch + kRows - 1) / kRows);
   const int grid = items < sm_count() ? items : sm_count();
-  absorb_o_tc_kernel<<<grid, kOThreads, smem, stream>>>(mf, mw, mo, batch, heads, err, 2000ull * 1000000ull);
-  return cudaGetLastError();
+  return launch_dependent(absorb_o_tc_kernel, grid, kOThreads, smem, stream, mf, mw, mo, batch, heads, err,
+                          2000ull * 1000000ull);
 }
 
 }  // namespace mla

@@ -16,6 +16,9 @@ __global__ void __launch_bounds__(kSchedThreads) schedule_kernel(const int32_t* 
   __shared__ int carry;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   grid_dep_launch_dependents();  // the decode grid may start its prologue now; it waits for this grid's writes
+  // Launched as a programmatic dependent of whatever ran before on the stream (which may
+  // have written the lengths, or still read this workspace): only the launch overlaps it.
+  grid_dep_wait();
   if (tid == 0) carry = 0;
   __syncthreads();
 
@@ -140,8 +143,16 @@ size_t carve_schedule(void* base, int batch, int heads, int num_workers, Schedul
 
 cudaError_t launch_schedule(const int32_t* seqlens, int batch, int max_blocks, int min_pages,
                             const Schedule& s, int* err, cudaStream_t stream) {
-  schedule_kernel<<<1, kSchedThreads, 0, stream>>>(seqlens, batch, max_blocks, min_pages, s, err);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(1, 1, 1);
+  cfg.blockDim = dim3(kSchedThreads, 1, 1);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, schedule_kernel, seqlens, batch, max_blocks, min_pages, s, err);
 }
 
 }  // namespace mla
