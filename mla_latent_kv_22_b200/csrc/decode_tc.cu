@@ -42,6 +42,11 @@
 // K-major B of QK^T and MN-major B of PV; 1 rope box [64 tokens x 32 dims], 64B
 // swizzle); a 24 KB send buffer and two 24 KB receive buffers.
 //
+// Several query tokens per sequence (decode_tc_kernel<true>): the rows are s_q query
+// tokens of hq heads each, read from and written to a per-sequence row stride with a row
+// offset (a launch handles at most 128 rows), and each row's valid columns end at its
+// query's causal window; a row (or a piece) that sees no token gets out 0, lse -inf.
+//
 // Every mbarrier wait is bounded by a time limit; on expiry the kernel records
 // MLA_ERR_DEVICE_TIMEOUT, tells the peer CTA to stop, drains its own TMA, bulk-copy
 // and MMA work, frees TMEM and returns.  No trap.
