@@ -520,18 +520,6 @@ bool map3d(CUtensorMap* m, CUtensorMapDataType t, const void* base, uint64_t d0,
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// Raise a kernel's dynamic shared memory limit once per device (outside any stream
-// capture that follows the first call on that device).
-cudaError_t allow_smem(const void* kernel, int bytes, bool (&done)[64]) {
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return e;
-  if (dev >= 0 && dev < 64 && done[dev]) return cudaSuccess;
-  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
-  if (e == cudaSuccess && dev >= 0 && dev < 64) done[dev] = true;
-  return e;
-}
-
 // Launch as a programmatic dependent of the previous grid on the stream.
 template <typename... Params, typename... Args>
 cudaError_t launch_dependent(void (*kernel)(Params...), int grid, int threads, int smem, cudaStream_t stream,
@@ -575,7 +563,7 @@ cudaError_t launch_absorb_q(const __nv_bfloat16* q_nope, const __nv_bfloat16* q_
     return cudaErrorInvalidValue;
   const int smem = kQSmem + 1024;
   static bool done[64] = {};
-  cudaError_t e = allow_smem(reinterpret_cast<const void*>(absorb_q_tc_kernel), smem, done);
+  cudaError_t e = allow_dynamic_smem(reinterpret_cast<const void*>(absorb_q_tc_kernel), smem, done);
   if (e != cudaSuccess) return e;
   const int items = heads * ((batch + kRows - 1) / kRows);
   const int grid = items < sm_count() ? items : sm_count();
@@ -596,7 +584,7 @@ cudaError_t launch_absorb_o(const float* out_latent, const __nv_bfloat16* w_uv, 
     return cudaErrorInvalidValue;
   const int smem = kOSmem + 1024;
   static bool done[64] = {};
-  cudaError_t e = allow_smem(reinterpret_cast<const void*>(absorb_o_tc_kernel), smem, done);
+  cudaError_t e = allow_dynamic_smem(reinterpret_cast<const void*>(absorb_o_tc_kernel), smem, done);
   if (e != cudaSuccess) return e;
   const int items = heads * ((batch + kRows - 1) / kRows);
   const int grid = items < sm_count() ? items : sm_count();

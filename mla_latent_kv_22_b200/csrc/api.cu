@@ -151,6 +151,17 @@ mla_status_t decode_plan(int heads, int* kernel, int* num_workers, int** err_wor
 
 mla_status_t record_error(mla_status_t s, const char* msg) { return fail(s, "%s", msg); }
 
+cudaError_t allow_dynamic_smem(const void* kernel, int bytes, bool (&done)[64]) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const bool tracked = dev >= 0 && dev < 64;
+  if (tracked && done[dev]) return cudaSuccess;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess && tracked) done[dev] = true;
+  return e;
+}
+
 int knob_value(int knob) { return (knob >= 0 && knob < 8) ? g_knobs[knob].load() : 0; }
 }  // namespace mla
 

@@ -238,12 +238,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_mma_kernel(DecodeArgs a) {
 int decode_mma_heads_per_cta() { return kHeadsPerCta; }
 
 cudaError_t launch_decode_mma(const DecodeArgs& a, cudaStream_t stream) {
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(decode_mma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  static bool done[64] = {};
+  cudaError_t e = allow_dynamic_smem(reinterpret_cast<const void*>(decode_mma_kernel), kSmemBytes, done);
+  if (e != cudaSuccess) return e;
   dim3 grid(a.sched.num_workers, (a.heads + kHeadsPerCta - 1) / kHeadsPerCta);
   decode_mma_kernel<<<grid, kThreads, kSmemBytes, stream>>>(a);
   return cudaGetLastError();

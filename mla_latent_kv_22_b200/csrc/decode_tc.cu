@@ -800,14 +800,10 @@ int decode_tc_max_workers(int sm_count) {
 }
 
 cudaError_t launch_decode_tc(const DecodeArgs& a, cudaStream_t stream) {
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(decode_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemAlloc);
-    if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(decode_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemAlloc);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  static bool done1[64] = {}, done2[64] = {};
+  cudaError_t e = allow_dynamic_smem(reinterpret_cast<const void*>(decode_tc_kernel<false>), kSmemAlloc, done1);
+  if (e == cudaSuccess) e = allow_dynamic_smem(reinterpret_cast<const void*>(decode_tc_kernel<true>), kSmemAlloc, done2);
+  if (e != cudaSuccess) return e;
   auto encode = get_encode();
   if (!encode) return cudaErrorNotSupported;
   // The cache as a 2-D tensor [rows, 576]: latent boxes of 64 dims (128B swizzle) and

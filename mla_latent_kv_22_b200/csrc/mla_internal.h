@@ -76,6 +76,11 @@ cudaError_t launch_absorb_q(const __nv_bfloat16* q_nope, const __nv_bfloat16* q_
 cudaError_t launch_absorb_o(const float* out_latent, const __nv_bfloat16* w_uv, float* out, int batch,
                             int heads, int* err, cudaStream_t stream);
 
+// Raises `kernel`'s dynamic shared memory limit to `bytes` on the current device, once
+// per device (the attribute belongs to the device's context); `done` is the caller's
+// per-device record.  Defined in api.cu.
+cudaError_t allow_dynamic_smem(const void* kernel, int bytes, bool (&done)[64]);
+
 // Defined in api.cu: the per-device decode plan, the thread's last-error text,
 // and raw knob values.
 mla_status_t decode_plan(int heads, int* kernel, int* num_workers, int** err_word);
