@@ -68,3 +68,31 @@ def test_algorithmic_bytes_headline():
     import bench
     assert bench.algorithmic_bytes(64, 128, 8192, 128) == 630_259_968
     assert bench.algorithmic_flops(64, 128, 8192) == 146_028_888_064
+
+
+def test_reference_arm_two_ranks_rank0_reports():
+    # Under torchrun with N > 1 the reference arm (the fp64 oracle) runs on rank 0 only:
+    # rank 0 prints one JSON line, every other rank exits 0 without output.
+    import json
+    procs = []
+    for r in range(2):
+        env = dict(os.environ, RANK=str(r), LOCAL_RANK=str(r), WORLD_SIZE="2", MASTER_ADDR="127.0.0.1",
+                   MASTER_PORT=str(_free_port()))
+        procs.append(subprocess.Popen([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                                       "--gpus", "2", "--steps", "1", "--warmup", "3"], env=env,
+                                      stdout=subprocess.PIPE, stderr=subprocess.PIPE, text=True, cwd=ROOT))
+    outs = []
+    for p in procs:
+        try:
+            out, err = p.communicate(timeout=300)
+        except subprocess.TimeoutExpired:
+            p.kill()
+            pytest.fail("reference arm did not finish")
+        assert p.returncode == 0, err
+        outs.append(out)
+    lines0 = [l for l in outs[0].splitlines() if l.startswith("{")]
+    assert len(lines0) == 1
+    rec = json.loads(lines0[0])
+    assert rec["impl"] == "reference" and rec["n_gpus"] == 2 and rec["value"] > 0
+    assert rec["e2e"]["h2d_bytes_per_step"] == 0 and rec["cpu_baseline"]["kind"] == "oracle"
+    assert not [l for l in outs[1].splitlines() if l.startswith("{")]
