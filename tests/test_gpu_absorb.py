@@ -17,7 +17,7 @@ def _f64(t):
     return t.double().cpu().numpy()
 
 
-@pytest.mark.parametrize("B,H", [(64, 128), (5, 3), (70, 16), (1, 1), (130, 32)])
+@pytest.mark.parametrize("B,H", [(64, 128), (5, 3), (70, 16), (1, 1), (130, 32), (300, 8)])
 def test_absorb_q(B, H):
     li = S.make_layer_inputs(B, H, seed=50 + B)
     qn, qr, wk = bf16_dev(li.q_nope), bf16_dev(li.q_rope), bf16_dev(li.w_uk)
@@ -31,7 +31,7 @@ def test_absorb_q(B, H):
     assert np.array_equal(got[..., 512:], ref[..., 512:])
 
 
-@pytest.mark.parametrize("B,H", [(64, 128), (5, 3), (70, 16), (130, 32)])
+@pytest.mark.parametrize("B,H", [(64, 128), (5, 3), (70, 16), (130, 32), (300, 8)])
 def test_absorb_o(B, H):
     li = S.make_layer_inputs(B, H, seed=60 + B)
     ol = torch.randn(B, H, 512, generator=torch.Generator().manual_seed(B)).mul_(0.05)
