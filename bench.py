@@ -12,7 +12,8 @@ steps stream the cache from HBM.
 
 With N > 1 it runs under torchrun, one replica per GPU (no data-path
 collective; the process group only times the job as the max over ranks).
-``--impl reference`` times the fp64 CPU oracle on the host cores instead.
+``--impl reference`` times the fp64 CPU oracle on the host cores instead, on whole steps
+of the same workload.
 """
 from __future__ import annotations
 
@@ -212,9 +213,17 @@ class ClockSampler:
 # CPU baseline: the fp64 oracle on a bounded sample of the workload.
 # ---------------------------------------------------------------------------
 
-def oracle_case_sample(n_seq: int):
+def headline_case():
+    """The timed workload's inputs (host arrays), the same for both arms."""
     import mla_synth as S
-    return S.make_decode_case(n_seq, H, T, seed=SEED, poison=False, latent_std=0.5, rope_std=1.0)
+    return S.config_case(3, headline=True, poison=False)
+
+
+def workload_config(world: int) -> dict:
+    """The `config` object of the JSON line; both arms print the same one."""
+    return {"workload": WORKLOAD, "global_batch": B * world, "seq_len": T, "heads": H, "page": PAGE,
+            "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+            "l2": "inputs larger than L2 (630 MB working set, 126 MB L2); no flush"}
 
 
 def blas_threads() -> int:
@@ -227,41 +236,40 @@ def blas_threads() -> int:
 
 
 def time_oracle_step(case) -> float:
-    """Seconds the oracle takes for all heads of the sample's sequences."""
+    """Seconds the oracle takes for one whole step: every sequence, every head."""
     import oracle as O
     t0 = time.perf_counter()
     O.mla_decode_ref(case.q, case.kv_cache, case.block_table, case.cache_seqlens, case.softmax_scale)
     return time.perf_counter() - t0
 
 
-def cpu_baseline(budget_s: float = 15.0) -> dict:
-    case = oracle_case_sample(1)
-    t1 = time_oracle_step(case)  # one sequence, all 128 heads
-    reps = max(1, min(64, int(budget_s / max(t1, 1e-3))))
+def cpu_baseline(case, budget_s: float = 15.0) -> dict:
+    """The oracle timed on whole steps of the workload (all 64 sequences, all heads)."""
+    t1 = time_oracle_step(case)
+    reps = max(3, min(20, int(budget_s / max(t1, 1e-3))))
     ts = [time_oracle_step(case) for _ in range(reps)]
-    per_seq = statistics.median(ts)
-    return {"value": per_seq * B * 1e6, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
-            "sample": f"fp64 numpy oracle on 1 of the 64 sequences (all 128 heads, T=8192), median of {reps} runs, "
-                      f"scaled x64 to the full step"}
+    return {"value": statistics.median(ts) * 1e6, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+            "sample": f"fp64 numpy oracle on the whole step (64 sequences x 128 heads, T=8192), "
+                      f"median of {reps} steps after one untimed step"}
 
 
 def run_reference(args) -> None:
     rank, _, world = dist_env()
     if world > 1 and rank != 0:
         return
-    case = oracle_case_sample(1)
+    case = headline_case()
     for _ in range(args.warmup):
         time_oracle_step(case)
     ts = [time_oracle_step(case) for _ in range(args.steps)]
-    us = statistics.mean(ts) * B * 1e6
+    us = statistics.mean(ts) * 1e6
     line = {
         "impl": "reference", "metric": METRIC, "value": us, "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": us / 1e3, "higher_is_better": False, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": WORKLOAD, "global_batch": B, "seq_len": T, "heads": H,
-                   "sample": "each step: 1 of 64 sequences, all heads; value scaled x64"},
+        "config": workload_config(world),
         "cpu_baseline": {"value": us, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
-                         "sample": "each step times the fp64 oracle on 1 of the 64 sequences, scaled x64"},
+                         "sample": "every step runs the fp64 oracle on the whole workload "
+                                   "(64 sequences x 128 heads, T=8192); mean over the timed steps"},
         "e2e": {"value": us, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -275,7 +283,6 @@ def run_ours(args) -> None:
     import torch
 
     import mla_latent_kv_22_b200 as M
-    import mla_synth as S
 
     rank, local_rank, world = dist_env()
     M.mla_set_knob("decode_kernel", {"auto": 0, "mma.sync": 1, "tcgen05": 2}[args.kernel])
@@ -283,7 +290,7 @@ def run_ours(args) -> None:
     device = torch.device("cuda", local_rank)
     dist = init_dist("nccl")
 
-    case = S.config_case(3, headline=True, poison=False)
+    case = headline_case()
     to_dev = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(device)
     q, kv = to_dev(case.q), to_dev(case.kv_cache)
     bt = torch.from_numpy(case.block_table).to(device)
@@ -408,9 +415,7 @@ def run_ours(args) -> None:
         "metric": METRIC, "value": us_step, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": False, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": WORKLOAD, "global_batch": B * world, "seq_len": T, "heads": H, "page": PAGE,
-                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
-                   "l2": "inputs larger than L2 (630 MB working set, 126 MB L2); no flush"},
+        "config": workload_config(world),
         "kv_tbps": B * T * D * 2 / (ms_step * 1e-3) / 1e12,
         "tflops": flops / (ms_step * 1e-3) / 1e12,
         "roofline_us": roofline_us,
@@ -427,7 +432,7 @@ def run_ours(args) -> None:
         "decode_kernel": kernel,
     }
     if world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline()
+        line["cpu_baseline"] = cpu_baseline(case)
     print(json.dumps(line), flush=True)
     if dist is not None:
         dist.destroy_process_group()

@@ -95,4 +95,8 @@ def test_reference_arm_two_ranks_rank0_reports():
     rec = json.loads(lines0[0])
     assert rec["impl"] == "reference" and rec["n_gpus"] == 2 and rec["value"] > 0
     assert rec["e2e"]["h2d_bytes_per_step"] == 0 and rec["cpu_baseline"]["kind"] == "oracle"
+    # both arms describe the workload with the same config object
+    sys.path.insert(0, ROOT)
+    import bench
+    assert rec["config"] == bench.workload_config(2)
     assert not [l for l in outs[1].splitlines() if l.startswith("{")]
