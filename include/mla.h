@@ -121,8 +121,7 @@ mla_status_t mla_decode(const void* q, const void* kv_cache, const int32_t* bloc
  * sequence sharing every load of its cached rows.
  * s_q >= 1, heads <= 128 and s_q * heads <= 2048, else MLA_ERR_UNSUPPORTED.
  * Up to 128 rows share one pass over the cache; more rows run as groups of 128,
- * each group reading the cache again.  It runs on the tcgen05 kernel only
- * (MLA_ERR_UNSUPPORTED if the kernel knob forces the other).  Every other
+ * each group reading the cache again.  Every other
  * argument, the workspace, determinism and error behaviour are those of
  * mla_decode (mla_workspace_size takes s_q * heads as its heads).
  */
@@ -214,15 +213,22 @@ const char* mla_last_error_message(void);
 typedef enum {
   MLA_KNOB_NUM_WORKERS = 0,     /* > 0: force the number of split workers; 0 = auto         */
   MLA_KNOB_MIN_PAGES = 1,       /* > 0: minimum pages per worker; 0 = auto                  */
-  MLA_KNOB_DECODE_KERNEL = 2,   /* 0 = auto, 1 = mma.sync kernel, 2 = tcgen05 kernel        */
+  MLA_KNOB_DECODE_KERNEL = 2,   /* 0 = auto (3); 2 = CTA pair split by latent dims, partial
+                                   scores exchanged through distributed shared memory;
+                                   3 = CTA pair split by heads, pair-wide tcgen05 MMAs       */
   MLA_KNOB_WAIT_LIMIT = 3,      /* > 0: time limit of bounded device waits in ms; 0 = 2000  */
-  MLA_KNOB_WITHHOLD_ARRIVE = 4  /* 1: the tcgen05 kernel's producer skips one arrive, so the
+  MLA_KNOB_WITHHOLD_ARRIVE = 4, /* 1: the decode kernel's producer skips one load, so the
                                    consumer's bounded wait must run out (timeout test)      */
+  MLA_KNOB_SPLIT_POLICY = 5     /* 0 = auto: one whole sequence per worker when batch <= the
+                                   worker count and the longest sequence is at most 16 pages
+                                   above the split quota, else split; 1 = always split;
+                                   2 = whole sequences whenever batch <= the worker count.
+                                   A forced MLA_KNOB_NUM_WORKERS always splits.             */
 } mla_knob_t;
 mla_status_t mla_set_knob(mla_knob_t knob, int value);
 int mla_get_knob(mla_knob_t knob);
 /* Which decode kernel mla_decode runs for `heads` under the current knobs:
-   1 = mma.sync kernel, 2 = tcgen05 kernel, -1 = none handles it. */
+   2 or 3 (MLA_KNOB_DECODE_KERNEL's numbering), -1 = none handles it. */
 int mla_selected_decode_kernel(int heads);
 
 /*

@@ -27,7 +27,7 @@ STATUS = {
     0: "MLA_OK", 1: "MLA_ERR_INVALID_ARG", 2: "MLA_ERR_UNSUPPORTED", 3: "MLA_ERR_WORKSPACE", 4: "MLA_ERR_CUDA",
     5: "MLA_ERR_DEVICE_BAD_PAGE", 6: "MLA_ERR_DEVICE_TIMEOUT",
 }
-KNOB = {"num_workers": 0, "min_pages": 1, "decode_kernel": 2, "wait_limit": 3, "withhold_arrive": 4}
+KNOB = {"num_workers": 0, "min_pages": 1, "decode_kernel": 2, "wait_limit": 3, "withhold_arrive": 4, "split_policy": 5}
 
 D_LATENT, D_ROPE, D_QK, PAGE, D_NOPE, D_V, MAX_HEADS = 512, 64, 576, 64, 128, 128, 128
 
@@ -229,7 +229,7 @@ def mla_get_knob(name: str) -> int:
 
 
 def mla_selected_decode_kernel(heads: int) -> int:
-    """1 = mma.sync kernel, 2 = tcgen05 kernel (what mla_decode runs for ``heads`` now)."""
+    """2 = dim-split pair kernel, 3 = head-split pair kernel (what mla_decode runs for ``heads`` now)."""
     return int(lib.mla_selected_decode_kernel(int(heads)))
 
 

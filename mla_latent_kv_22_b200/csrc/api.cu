@@ -14,13 +14,6 @@
 #include "mla.h"
 #include "mla_internal.h"
 
-namespace mla {
-// Defined in decode_tc.cu.
-cudaError_t launch_decode_tc(const DecodeArgs& a, cudaStream_t stream);
-bool decode_tc_supported(int heads);
-int decode_tc_max_workers(int sm_count);
-}
-
 namespace {
 
 using namespace mla;
@@ -81,20 +74,21 @@ mla_status_t device_state(DeviceState** out) {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-// Decode kernel choice: knob, else the tcgen05 kernel when it handles the shape.
+// Decode kernel choice: the knob (2 = dim-split pair, 3 = head-split pair), else the
+// head-split pair kernel.  Both handle 1..128 rows per launch.
 int pick_kernel(int heads) {
+  if (heads < 1 || heads > MLA_MAX_HEADS) return -1;
   const int k = g_knobs[MLA_KNOB_DECODE_KERNEL].load();
-  if (k == 1) return 1;
-  if (k == 2) return decode_tc_supported(heads) ? 2 : -1;
-  return decode_tc_supported(heads) ? 2 : 1;
+  if (k == 0) return 3;
+  return (k == 2 || k == 3) ? k : -1;
 }
 
 int num_workers_for(const DeviceState& d, int kernel, int heads) {
+  (void)heads;
   const int forced = g_knobs[MLA_KNOB_NUM_WORKERS].load();
   if (forced > 0) return forced;
-  if (kernel == 2) return std::max(1, std::min(d.sm_count / 2, decode_tc_max_workers(d.sm_count)));  // CTA pairs
-  const int groups = (heads + decode_mma_heads_per_cta() - 1) / decode_mma_heads_per_cta();
-  return std::max(1, d.sm_count / groups);
+  const int occ = kernel == 2 ? decode_tc_max_workers(d.sm_count) : decode_pair_max_workers(d.sm_count);
+  return std::max(1, std::min(d.sm_count / 2, occ));  // CTA pairs
 }
 
 mla_status_t ensure_workspace(DeviceState& d, size_t need, cudaStream_t stream) {
@@ -150,6 +144,31 @@ mla_status_t decode_plan(int heads, int* kernel, int* num_workers, int** err_wor
 }
 
 mla_status_t record_error(mla_status_t s, const char* msg) { return fail(s, "%s", msg); }
+
+cudaError_t launch_decode(int kernel, const DecodeArgs& a, cudaStream_t stream) {
+  return kernel == 2 ? launch_decode_tc(a, stream) : launch_decode_pair(a, stream);
+}
+
+int decode_granule(int kernel) { return kernel == 3 ? 4 : 1; }
+
+int schedule_whole_slack() {
+  if (g_knobs[MLA_KNOB_NUM_WORKERS].load() > 0) return -1;
+  const int v = g_knobs[MLA_KNOB_SPLIT_POLICY].load();
+  return v == 0 ? 16 : v == 1 ? -1 : 1 << 30;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    cudaDriverEntryPointQueryResult q;
+    void* p = nullptr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
 
 cudaError_t allow_dynamic_smem(const void* kernel, int bytes, bool (&done)[64]) {
   int dev = 0;
@@ -288,7 +307,6 @@ mla_status_t decode_call(const void* q, const void* kv_cache, const int32_t* blo
   const int group = std::min(heads, (int)MLA_MAX_HEADS);  // rows per launch
   const int kernel = pick_kernel(group);
   if (kernel < 0) return fail(MLA_ERR_UNSUPPORTED, "requested decode kernel does not handle heads = %d", heads);
-  if (s_q > 1 && kernel != 2) return fail(MLA_ERR_UNSUPPORTED, "several query tokens need the tcgen05 kernel");
   const int P = num_workers_for(*d, kernel, group);
   const size_t need = carve_schedule(nullptr, batch, group, P, nullptr);
   s = ensure_workspace(*d, need, stream);
@@ -317,13 +335,14 @@ mla_status_t decode_call(const void* q, const void* kv_cache, const int32_t* blo
   const int min_pages = g_knobs[MLA_KNOB_MIN_PAGES].load() > 0 ? g_knobs[MLA_KNOB_MIN_PAGES].load() : 4;
 
   record_event(*d, 0, stream);
-  cudaError_t e = launch_schedule(cache_seqlens, batch, max_blocks, min_pages, a.sched, d->err, stream);
+  cudaError_t e = launch_schedule(cache_seqlens, batch, max_blocks, min_pages, decode_granule(kernel),
+                                  schedule_whole_slack(), a.sched, d->err, stream);
   if (e != cudaSuccess) return cuda_fail(e, "schedule launch");
   record_event(*d, 1, stream);
   for (int r0 = 0; r0 < heads; r0 += group) {
     a.row0 = r0;
     a.heads = std::min(group, heads - r0);
-    e = kernel == 2 ? launch_decode_tc(a, stream) : launch_decode_mma(a, stream);
+    e = launch_decode(kernel, a, stream);
     if (e != cudaSuccess) return cuda_fail(e, "decode launch");
     if (r0 + group >= heads) record_event(*d, 2, stream);
     e = launch_combine(a, stream);

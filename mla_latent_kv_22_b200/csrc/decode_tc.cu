@@ -53,8 +53,6 @@
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
-#include <mutex>
-
 #include "mla_device.cuh"
 #include "mla_internal.h"
 #include "sm100_ptx.cuh"
@@ -766,26 +764,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   }
 }
 
-PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    cudaDriverEntryPointQueryResult q;
-    void* p = nullptr;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-  });
-  return fn;
-}
-
 }  // namespace
 
-bool decode_tc_supported(int heads) { return heads >= 1 && heads <= 128; }
-
 int decode_tc_max_workers(int sm_count) {
-  static int cached = -1;
-  if (cached < 0) {
+  static int cached_dev[64];
+  static bool have[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) dev = 0;
+  if (!have[dev]) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(2 * (sm_count / 2), 1, 1);
     cfg.blockDim = dim3(kThreads, 1, 1);
@@ -794,9 +780,10 @@ int decode_tc_max_workers(int sm_count) {
     int clusters = 0;
     if (cudaOccupancyMaxActiveClusters(&clusters, decode_tc_kernel<false>, &cfg) != cudaSuccess || clusters <= 0)
       clusters = sm_count / 2;
-    cached = clusters;
+    cached_dev[dev] = clusters;
+    have[dev] = true;
   }
-  return cached;
+  return cached_dev[dev];
 }
 
 cudaError_t launch_decode_tc(const DecodeArgs& a, cudaStream_t stream) {
@@ -804,7 +791,7 @@ cudaError_t launch_decode_tc(const DecodeArgs& a, cudaStream_t stream) {
   cudaError_t e = allow_dynamic_smem(reinterpret_cast<const void*>(decode_tc_kernel<false>), kSmemAlloc, done1);
   if (e == cudaSuccess) e = allow_dynamic_smem(reinterpret_cast<const void*>(decode_tc_kernel<true>), kSmemAlloc, done2);
   if (e != cudaSuccess) return e;
-  auto encode = get_encode();
+  auto encode = tensor_map_encoder();
   if (!encode) return cudaErrorNotSupported;
   // The cache as a 2-D tensor [rows, 576]: latent boxes of 64 dims (128B swizzle) and
   // rope boxes of 32 dims (64B swizzle), 64 rows (one page) each.

@@ -6,6 +6,8 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include <cudaTypedefs.h>
+
 #include "mla.h"
 
 namespace mla {
@@ -65,10 +67,14 @@ struct DecodeArgs {
   int s_q, hq, row_stride, row0;
 };
 
-cudaError_t launch_schedule(const int32_t* seqlens, int batch, int max_blocks, int min_pages,
-                            const Schedule& s, int* err, cudaStream_t stream);
-cudaError_t launch_decode_mma(const DecodeArgs& a, cudaStream_t stream);
-int decode_mma_heads_per_cta();
+// granule: the pages per worker are rounded up to a multiple of it (the pair kernel
+// walks its range in steps of 4 pages).  whole_slack >= 0: one whole sequence per worker
+// when batch <= workers and the longest sequence exceeds the split quota by at most
+// whole_slack pages; < 0: always split.
+cudaError_t launch_schedule(const int32_t* seqlens, int batch, int max_blocks, int min_pages, int granule,
+                            int whole_slack, const Schedule& s, int* err, cudaStream_t stream);
+// The whole-sequence slack for the current knobs (a forced worker count always splits).
+int schedule_whole_slack();
 cudaError_t launch_combine(const DecodeArgs& a, cudaStream_t stream);
 cudaError_t launch_absorb_q(const __nv_bfloat16* q_nope, const __nv_bfloat16* q_rope,
                             const __nv_bfloat16* w_uk, __nv_bfloat16* q_out, int batch, int heads, int* err,
@@ -86,6 +92,19 @@ cudaError_t allow_dynamic_smem(const void* kernel, int bytes, bool (&done)[64]);
 mla_status_t decode_plan(int heads, int* kernel, int* num_workers, int** err_word);
 mla_status_t record_error(mla_status_t s, const char* msg);
 int knob_value(int knob);
+
+// Decode kernels (mla_selected_decode_kernel's numbering): 2 = the CTA pair split by
+// dims with partial scores exchanged through distributed shared memory
+// (decode_tc.cu), 3 = the CTA pair split by heads with pair-wide MMAs (decode_pair.cu).
 cudaError_t launch_decode_tc(const DecodeArgs& a, cudaStream_t stream);
+int decode_tc_max_workers(int sm_count);
+cudaError_t launch_decode_pair(const DecodeArgs& a, cudaStream_t stream);
+int decode_pair_max_workers(int sm_count);
+// The launch of kernel `kernel` and its page granule of the schedule.
+cudaError_t launch_decode(int kernel, const DecodeArgs& a, cudaStream_t stream);
+int decode_granule(int kernel);
+
+// cuTensorMapEncodeTiled from the driver (resolved once; null if unavailable).  Defined in api.cu.
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder();
 
 }  // namespace mla

@@ -122,9 +122,10 @@ extern "C" mla_status_t mla_decode_noalloc(const void* q, const void* kv_cache, 
   const int mp = mla::knob_value(MLA_KNOB_MIN_PAGES);
   const int min_pages = mp > 0 ? mp : 4;
 
-  e = mla::launch_schedule(cache_seqlens, batch, max_blocks, min_pages, a.sched, err, stream);
+  e = mla::launch_schedule(cache_seqlens, batch, max_blocks, min_pages, mla::decode_granule(kernel),
+                           mla::schedule_whole_slack(), a.sched, err, stream);
   if (e != cudaSuccess) return reject(MLA_ERR_CUDA, "schedule launch failed");
-  e = kernel == 2 ? mla::launch_decode_tc(a, stream) : mla::launch_decode_mma(a, stream);
+  e = mla::launch_decode(kernel, a, stream);
   if (e != cudaSuccess) return reject(MLA_ERR_CUDA, "decode launch failed");
   e = mla::launch_combine(a, stream);
   if (e != cudaSuccess) return reject(MLA_ERR_CUDA, "combine launch failed");

@@ -10,16 +10,20 @@ namespace {
 constexpr int kSchedThreads = 1024;
 
 __global__ void __launch_bounds__(kSchedThreads) schedule_kernel(const int32_t* __restrict__ seqlens, int B,
-                                                                 int max_blocks, int min_pages, Schedule s,
-                                                                 int* err) {
+                                                                 int max_blocks, int min_pages, int granule,
+                                                                 int whole_slack, Schedule s, int* err) {
   __shared__ int warp_sums[kSchedThreads / 32];
   __shared__ int carry;
+  __shared__ int max_pages;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   grid_dep_launch_dependents();  // the decode grid may start its prologue now; it waits for this grid's writes
   // Launched as a programmatic dependent of whatever ran before on the stream (which may
   // have written the lengths, or still read this workspace): only the launch overlaps it.
   grid_dep_wait();
-  if (tid == 0) carry = 0;
+  if (tid == 0) {
+    carry = 0;
+    max_pages = 0;
+  }
   __syncthreads();
 
   // 1. Exclusive prefix sum of pages per sequence, 1024 sequences per pass.  With a
@@ -59,6 +63,7 @@ __global__ void __launch_bounds__(kSchedThreads) schedule_kernel(const int32_t* 
     __syncthreads();
     const int incl = x + (warp ? warp_sums[warp - 1] : 0) + carry;
     if (b < B) s.seq_start[b] = incl - n;
+    if (n > 0) atomicMax(&max_pages, n);
     my_start = incl - n;
     my_n = n;
     my_bad = bad;
@@ -74,7 +79,33 @@ __global__ void __launch_bounds__(kSchedThreads) schedule_kernel(const int32_t* 
   int q = (N + P - 1) / P;
   if (q < min_pages) q = min_pages;
   if (q < 1) q = 1;
+  q = (q + granule - 1) / granule * granule;
   if (tid == 0) *s.quota = q;
+
+  // Whole sequences, one per worker, when there are no more sequences than workers and
+  // the longest costs at most whole_slack pages more than the split quota: a split
+  // sequence pays for a piece boundary in its workers and for the combine, so nearly
+  // uniform lengths run faster unsplit (whole_slack < 0: always split).
+  if (whole_slack >= 0 && B <= P && max_pages <= q + whole_slack) {
+    for (int w = tid; w < P; w += kSchedThreads) {
+      int n = 0;
+      if (w < B) {
+        const int T = seqlens[w];
+        n = (T < 0 || T > max_blocks * kPage) ? 0 : (T + kPage - 1) / kPage;
+      }
+      s.ranges[w] = n > 0 ? WorkerRange{w, 0, w, n} : WorkerRange{-1, 0, -1, 0};
+    }
+    for (int b = tid; b < B; b += kSchedThreads) {
+      const int T = seqlens[b];
+      const bool bad = T < 0 || T > max_blocks * kPage;
+      SeqInfo si;
+      si.first_worker = b;
+      si.num_pieces = bad ? -1 : (T > 0 ? 1 : 0);
+      si.first_slot = b;
+      s.seq[b] = si;
+    }
+    return;
+  }
 
   // 2. Workers past the last page have no work.
   for (int w = tid; w < P; w += kSchedThreads)
@@ -141,8 +172,8 @@ size_t carve_schedule(void* base, int batch, int heads, int num_workers, Schedul
   return off;
 }
 
-cudaError_t launch_schedule(const int32_t* seqlens, int batch, int max_blocks, int min_pages,
-                            const Schedule& s, int* err, cudaStream_t stream) {
+cudaError_t launch_schedule(const int32_t* seqlens, int batch, int max_blocks, int min_pages, int granule,
+                            int whole_slack, const Schedule& s, int* err, cudaStream_t stream) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(1, 1, 1);
   cfg.blockDim = dim3(kSchedThreads, 1, 1);
@@ -152,7 +183,8 @@ cudaError_t launch_schedule(const int32_t* seqlens, int batch, int max_blocks, i
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, schedule_kernel, seqlens, batch, max_blocks, min_pages, s, err);
+  return cudaLaunchKernelEx(&cfg, schedule_kernel, seqlens, batch, max_blocks, min_pages, granule < 1 ? 1 : granule,
+                            whole_slack, s, err);
 }
 
 }  // namespace mla

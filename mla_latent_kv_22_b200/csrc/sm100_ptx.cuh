@@ -39,6 +39,18 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
+// try_wait with CTA-scope acquire: enough for a barrier that only tensor-memory-access
+// (TMA) transactions and MMA commits complete, whose data the async proxy then reads.
+__device__ __forceinline__ bool mbar_try_wait_cta(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2;\n"
+      " selp.b32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
 // try_wait with a suspend-time hint (ns): the thread sleeps until the phase completes
 // or the hint expires, whichever is first.
 __device__ __forceinline__ bool mbar_try_wait_hint(uint32_t bar, uint32_t parity, uint32_t hint_ns) {
@@ -170,6 +182,12 @@ __device__ __forceinline__ uint64_t desc_sw128(uint32_t addr, uint32_t lbo_bytes
   d |= (uint64_t)2 << 61;
   return d;
 }
+// The address-independent bits of a 128B-swizzle descriptor: OR in (addr >> 4) (14 bits,
+// shared memory is below 256 KB), and step the start address by adding bytes / 16.
+__host__ __device__ constexpr uint64_t desc_sw128_const(uint32_t lbo_bytes, uint32_t sbo_bytes) {
+  return ((uint64_t)((lbo_bytes >> 4) & 0x3FFFu) << 16) | ((uint64_t)((sbo_bytes >> 4) & 0x3FFFu) << 32) |
+         ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
+}
 // Same with 64-byte swizzle (mode 4): 64-byte rows, 8-row atoms of 512 bytes.
 __device__ __forceinline__ uint64_t desc_sw64(uint32_t addr, uint32_t lbo_bytes, uint32_t sbo_bytes) {
   uint64_t d = 0;
@@ -220,6 +238,98 @@ __device__ __forceinline__ void bulk_copy_to_peer(uint32_t dst_cluster, uint32_t
 }
 __device__ __forceinline__ void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
 __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
+
+// ---------------------------------------------------------------- pair-wide (cta_group::2) forms
+// A pair of CTAs (a 2-CTA cluster) allocates the same tensor-memory columns in both SMs;
+// one warp of each CTA executes these, with the same destination shared-memory offset.
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t dst_smem, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst_smem), "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish_pair() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+// Pair-wide MMA, issued by the even CTA of the pair: each CTA supplies half of A's rows
+// and half of B's N columns at the same shared-memory offsets, and receives its rows of D.
+__device__ __forceinline__ void mma_pair_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                            uint32_t accumulate) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(
+          d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// Four pair-wide MMAs along K (descriptors stepped by `a_step` / `b_step` 16-byte units),
+// issued by one elected lane of a converged warp: the whole warp runs the issue loop
+// (uniform control flow keeps the descriptors in the uniform datapath) and one lane
+// issues.  The first MMA accumulates iff `accumulate`, the other three always.
+template <uint32_t kAStep, uint32_t kBStep>
+__device__ __forceinline__ void mma_pair_x4_elect(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                                  uint32_t accumulate) {
+  asm volatile(
+      "{\n .reg .pred acc, one, e;\n .reg .b64 a1, a2, a3, b1, b2, b3;\n"
+      " setp.ne.b32 acc, %4, 0;\n setp.eq.u32 one, 1, 1;\n elect.sync _|e, 0xffffffff;\n"
+      " add.u64 a1, %1, %5;\n add.u64 a2, %1, %6;\n add.u64 a3, %1, %7;\n"
+      " add.u64 b1, %2, %8;\n add.u64 b2, %2, %9;\n add.u64 b3, %2, %10;\n"
+      " @e tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, acc;\n"
+      " @e tcgen05.mma.cta_group::2.kind::f16 [%0], a1, b1, %3, one;\n"
+      " @e tcgen05.mma.cta_group::2.kind::f16 [%0], a2, b2, %3, one;\n"
+      " @e tcgen05.mma.cta_group::2.kind::f16 [%0], a3, b3, %3, one;\n}\n" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "n"(kAStep), "n"(2 * kAStep), "n"(3 * kAStep),
+      "n"(kBStep), "n"(2 * kBStep), "n"(3 * kBStep)
+      : "memory");
+}
+// The same with A in tensor memory (pair-wide layout: each CTA holds its rows of A in
+// lanes 0-63 and again in lanes 64-127), stepped by 8 columns (16 bf16) along K.
+template <uint32_t kBStep>
+__device__ __forceinline__ void mma_pair_ts_x4_elect(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                                     uint32_t accumulate) {
+  asm volatile(
+      "{\n .reg .pred acc, one, e;\n .reg .b32 a1, a2, a3;\n .reg .b64 b1, b2, b3;\n"
+      " setp.ne.b32 acc, %4, 0;\n setp.eq.u32 one, 1, 1;\n elect.sync _|e, 0xffffffff;\n"
+      " add.u32 a1, %1, 8;\n add.u32 a2, %1, 16;\n add.u32 a3, %1, 24;\n"
+      " add.u64 b1, %2, %5;\n add.u64 b2, %2, %6;\n add.u64 b3, %2, %7;\n"
+      " @e tcgen05.mma.cta_group::2.kind::f16 [%0], [%1], %2, %3, acc;\n"
+      " @e tcgen05.mma.cta_group::2.kind::f16 [%0], [a1], b1, %3, one;\n"
+      " @e tcgen05.mma.cta_group::2.kind::f16 [%0], [a2], b2, %3, one;\n"
+      " @e tcgen05.mma.cta_group::2.kind::f16 [%0], [a3], b3, %3, one;\n}\n" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate), "n"(kBStep), "n"(2 * kBStep), "n"(3 * kBStep)
+      : "memory");
+}
+// mma_commit_pair from one elected lane of a converged warp.
+__device__ __forceinline__ void mma_commit_pair_elect(uint32_t bar, uint16_t cta_mask) {
+  asm volatile(
+      "{\n .reg .pred e;\n elect.sync _|e, 0xffffffff;\n"
+      " @e tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;\n}\n" ::"r"(
+          bar),
+      "h"(cta_mask)
+      : "memory");
+}
+// Arrive on the mbarrier at shared-memory offset `bar` of every CTA in `cta_mask` once
+// all pair-wide tcgen05 operations issued so far by this thread are complete.
+__device__ __forceinline__ void mma_commit_pair(uint32_t bar, uint16_t cta_mask) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(bar),
+      "h"(cta_mask)
+      : "memory");
+}
+// 2-D tiled load into this CTA's shared memory whose byte count completes on an mbarrier
+// of the pair (`bar_cluster`, a cluster address, e.g. the even CTA's barrier).  No multicast.
+__device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const void* map, int x, int y, uint32_t bar_cluster) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], "
+      "[%4];" ::"r"(dst),
+      "l"(map), "r"(x), "r"(y), "r"(bar_cluster)
+      : "memory");
+}
+// Named barrier over `nthreads` threads (a multiple of 32) of this CTA.
+__device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t nthreads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
 
 }  // namespace sm100
 }  // namespace mla

@@ -23,7 +23,7 @@ def main() -> None:
     ap.add_argument("--heads", type=int, default=128)
     ap.add_argument("--seqlen", type=int, default=4096)
     ap.add_argument("--steps", type=int, default=3)
-    ap.add_argument("--kernel", type=int, default=0, help="0 auto, 1 mma.sync, 2 tcgen05")
+    ap.add_argument("--kernel", type=int, default=0, help="0 auto, 2 dim-split pair, 3 head-split pair")
     ap.add_argument("--absorb", action="store_true", help="run the two absorption GEMMs instead")
     a = ap.parse_args()
     if a.absorb:

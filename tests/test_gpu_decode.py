@@ -24,12 +24,14 @@ def oracle_for(case, batch=None, heads=None):
                             batch=batch, heads=heads)
 
 
-@pytest.fixture(autouse=True, params=[1, 2], ids=["mma", "tcgen05"])
+@pytest.fixture(autouse=True, params=[2, 3], ids=["dimsplit", "pair"])
 def kernel(request):
-    """Every test runs on both decode kernels."""
+    """Every test runs on both decode kernels: 2 = the CTA pair split by latent dims
+    (partial scores exchanged through distributed shared memory), 3 = the CTA pair
+    split by heads (pair-wide MMAs)."""
     M.mla_set_knob("decode_kernel", request.param)
     yield request.param
-    for k in ("num_workers", "min_pages", "decode_kernel", "wait_limit", "withhold_arrive"):
+    for k in ("num_workers", "min_pages", "decode_kernel", "wait_limit", "withhold_arrive", "split_policy"):
         M.mla_set_knob(k, 0)
 
 

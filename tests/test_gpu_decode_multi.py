@@ -20,9 +20,11 @@ from gpu_helpers import assert_close, upload
 pytestmark = pytest.mark.gpu
 
 
-@pytest.fixture(autouse=True)
-def _reset_knobs():
-    yield
+@pytest.fixture(autouse=True, params=[2, 3], ids=["dimsplit", "pair"])
+def kernel(request):
+    """Every test runs on both decode kernels."""
+    M.mla_set_knob("decode_kernel", request.param)
+    yield request.param
     for k in ("num_workers", "min_pages", "decode_kernel"):
         M.mla_set_knob(k, 0)
 
@@ -109,7 +111,7 @@ def test_multi_rejects_what_it_does_not_handle():
     with pytest.raises(M.MlaError) as ei:
         M.mla_decode_multi(too_many, dev[1], dev[2], dev[3], out, lse, c.softmax_scale)
     assert ei.value.name == "MLA_ERR_UNSUPPORTED"
-    M.mla_set_knob("decode_kernel", 1)  # the mma.sync kernel has no causal rows
+    M.mla_set_knob("decode_kernel", 1)  # names no decode kernel
     with pytest.raises(M.MlaError) as ei:
         _run(c, q, 2, 64, dev)
     assert ei.value.name == "MLA_ERR_UNSUPPORTED"
