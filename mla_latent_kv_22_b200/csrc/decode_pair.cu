@@ -384,8 +384,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       // Descriptors are built once per operand tile and stepped along K by constant adds
       // (a K-major step of 16 dims is 32 bytes, an MN-major step of 16 tokens 2048 bytes).
       constexpr uint64_t kKMajor = desc_sw128_const(16, 1024), kMNMajor = desc_sw128_const(8192, 1024);
-      const uint64_t dq0 = kKMajor | ((sbase + kOffQ) >> 4), dp0 = kKMajor | ((sbase + kOffP) >> 4);
-      const uint32_t ring4 = (sbase + kOffRing) >> 4;
+      const uint64_t dq0 = kKMajor | desc_addr(sbase + kOffQ), dp0 = kKMajor | desc_addr(sbase + kOffP);
+      const uint32_t ring4 = desc_addr(sbase + kOffRing);
       // The ring position as a slot index and a phase bit.  The value slot of a ragged
       // last page also waits for both CTAs to have zeroed its rows past the sequence end;
       // kTReady completes once per such page, `tails` counts them.

@@ -182,8 +182,11 @@ __device__ __forceinline__ uint64_t desc_sw128(uint32_t addr, uint32_t lbo_bytes
   d |= (uint64_t)2 << 61;
   return d;
 }
-// The address-independent bits of a 128B-swizzle descriptor: OR in (addr >> 4) (14 bits,
-// shared memory is below 256 KB), and step the start address by adding bytes / 16.
+// The start-address field of a descriptor: the 14-bit 16-byte index within this CTA's
+// shared memory (a shared-window address may carry more than the CTA-local offset).
+__device__ __forceinline__ uint32_t desc_addr(uint32_t smem_addr) { return (smem_addr & 0x3FFFFu) >> 4; }
+// The address-independent bits of a 128B-swizzle descriptor: OR in desc_addr(addr), and
+// step the start address by adding bytes / 16.
 __host__ __device__ constexpr uint64_t desc_sw128_const(uint32_t lbo_bytes, uint32_t sbo_bytes) {
   return ((uint64_t)((lbo_bytes >> 4) & 0x3FFFu) << 16) | ((uint64_t)((sbo_bytes >> 4) & 0x3FFFu) << 32) |
          ((uint64_t)1 << 46) | ((uint64_t)2 << 61);

@@ -3,9 +3,10 @@
 under stream capture, paths that cannot absorb cudaMalloc's device sync).  It uses
 the library's static device scratch instead of the workspace.
 
-Checked through the C ABI against mla_decode on two calls in a row with different
-inputs (the scratch keeps the previous call's contents, so a stale read would
-show), within the tolerances the other GPU tests use.  This file is collected last
+Checked through the C ABI against the fp64 oracle (mla_decode_ref) and against
+mla_decode, on two calls in a row with different inputs (the scratch keeps the
+previous call's contents, so a stale read would show), within the tolerances the
+other GPU tests use.  This file is collected last
 so that a run stopping at the first failure has run every other test already.
 """
 import ctypes
@@ -16,7 +17,8 @@ import torch
 
 import mla_latent_kv_22_b200 as M
 import mla_synth as S
-from gpu_helpers import LSE_ATOL, OUT_ATOL, OUT_RTOL, upload
+import oracle as O
+from gpu_helpers import LSE_ATOL, OUT_ATOL, OUT_RTOL, assert_close, upload
 
 pytestmark = pytest.mark.gpu
 
@@ -43,20 +45,26 @@ def _close(a, b):
     assert np.abs(al - bl).max() <= LSE_ATOL
 
 
-def test_noalloc_matches_mla_decode_on_two_calls_in_a_row():
+def _oracle(case):
+    return O.mla_decode_ref(case.q, case.kv_cache, case.block_table, case.cache_seqlens, case.softmax_scale)
+
+
+def test_noalloc_matches_oracle_and_mla_decode_on_two_calls_in_a_row():
     cases = [S.make_decode_case(16, 128, S.uniform_seqlens(3, 16, 100, 4000), seed=71, poison=True),
              S.make_decode_case(5, 128, [4096, 1, 64, 65, 3000], seed=72, poison=True)]
-    for case in cases:
+    for i, case in enumerate(cases):
         dev = upload(case)
-        ref = _call(M.lib.mla_decode, case, dev)
         got = _call(M.lib.mla_decode_noalloc, case, dev)
-        _close(got, ref)
+        assert_close(*got, *_oracle(case), what=f"noalloc case {i} vs oracle")
+        _close(got, _call(M.lib.mla_decode, case, dev))
 
 
 def test_noalloc_contiguous_and_few_heads():
     case = S.make_decode_case(3, 16, [700, 64, 1], seed=73, paged=False, poison=True)
     dev = upload(case)
-    _close(_call(M.lib.mla_decode_noalloc, case, dev), _call(M.lib.mla_decode, case, dev))
+    got = _call(M.lib.mla_decode_noalloc, case, dev)
+    assert_close(*got, *_oracle(case), what="noalloc contiguous vs oracle")
+    _close(got, _call(M.lib.mla_decode, case, dev))
 
 
 def test_noalloc_rejects_sizes_beyond_its_scratch():
