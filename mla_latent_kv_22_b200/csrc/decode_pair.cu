@@ -16,18 +16,21 @@
 // every row the pair fetched for the scores; that second read hits L2 (the rows were
 // fetched a few microseconds earlier), so HBM sees every cached byte once.
 //
-// Accumulator layout (pair-wide M = 128: 64 rows per CTA, the N columns split in two
-// halves over TMEM lanes 0-63 and 64-127).  In CTA r, lane l < 64 holds head 64r + l and
-// the first half of the columns, lane l >= 64 holds head 64r + l - 64 and the second:
-//   TMEM [0, 256)   O: block j = [128j, 128j+128) holds dims [256j, 256j+128) in lanes
-//                   0-63 and dims [256j+128, 256j+256) in lanes 64-127
-//   TMEM [256, 512) two S buffers of 128 columns: tokens [0,128) of the step in lanes
-//                   0-63, tokens [128,256) in lanes 64-127
-// Shared memory (per CTA): q' of the CTA's 64 heads (9 boxes of [64 rows x 64 dims],
-// 128B swizzle: the A operand of QK^T, 72 KB), P of its heads (4 boxes of [64 rows x
-// 64 tokens]: the A operand of PV, 32 KB), and a ring of 7 slots of two boxes (16 KB):
-// a score slot holds one 64-dim column block of the CTA's two pages (the 128-row
-// K-major B tile), a value slot holds 128 dims of one page (the MN-major B tile).
+// Tensor memory (pair-wide M = 128: 64 rows per CTA, the N columns of an accumulator
+// split in two halves over TMEM lanes 0-63 and 64-127).  In CTA r, lane l < 64 holds
+// head 64r + l and the first half of the columns, lane l >= 64 holds head 64r + l - 64
+// and the second:
+//   [0, 256)    O: block j = [128j, 128j+128) holds dims [256j, 256j+128) in lanes
+//               0-63 and dims [256j+128, 256j+256) in lanes 64-127
+//   [256, 384)  S of one step: tokens [0,128) in lanes 0-63, [128,256) in lanes 64-127
+//   [384, 512)  q' dims [0, 256) as the A operand of the first score MMAs (the pair-wide
+//               A layout: lanes l and l + 64 both hold head 64r + (l & 63))
+// Shared memory (per CTA): q' dims [256, 576) of the CTA's 64 heads (5 boxes of [64
+// rows x 64 dims], 128B swizzle, 40 KB), P of its heads (4 boxes of [64 rows x 64
+// tokens]: the A operand of PV, 32 KB), and a ring of 4 slots of four boxes (32 KB): a
+// score slot holds two 64-dim column blocks of the CTA's two pages (two 128-row
+// K-major B tiles; the rope slot only one), a value slot the CTA's two 128-dim halves
+// of one page (MN-major B tiles).
 //
 // Roles (384 threads per CTA).  Warp 0: TMA producer (q' per piece, then the ring in
 // the order the MMAs consume it: scores of step i, then values of step i-1).  Warp 1: TMEM allocation; in CTA 0 the MMA
