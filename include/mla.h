@@ -93,7 +93,7 @@ enum {
  *               scales by 1/sqrt(d_k + d_r)).
  * Rows of a last page beyond T_b, and unused block-table entries, may hold
  * anything (NaN included); they do not affect the result.
- * Uses the library workspace (split partials and schedule): see
+ * Uses the library workspace (split partials and per-sequence records): see
  * mla_workspace_size / mla_set_workspace.  The split of each sequence depends
  * only on (batch, heads, cache_seqlens, the device's SM count), never on page
  * ids, so a paged and a contiguous cache holding the same rows give
@@ -163,16 +163,15 @@ mla_status_t mla_absorb_o(const float* out_latent, const void* w_uv, float* out,
  *
  * The pages have no counterpart of this call; it exists for callers such as a
  * serving runtime that has already reserved all device memory for its own pool,
- * code running while a stream is captured into a CUDA graph (where cudaMalloc is
- * not allowed), or latency-critical paths that cannot absorb cudaMalloc's implicit
- * device synchronisation.  Arguments, layouts, results and errors are those of
+ * or latency-critical paths that cannot absorb cudaMalloc's implicit device
+ * synchronisation.  Arguments, layouts, results and errors are those of
  * mla_decode.  Instead of the workspace, it uses one 32 MiB static device array
  * that each GPU loading the library holds until exit; it never calls cudaMalloc or
- * cudaFree.  Sizes whose split partials and schedule do not fit are rejected with
- * MLA_ERR_UNSUPPORTED before any launch; to fit, it may split over fewer workers
+ * cudaFree.  Sizes whose split partials and per-sequence records do not fit are
+ * rejected with MLA_ERR_UNSUPPORTED before any launch; to fit, it may split over fewer workers
  * than mla_decode, so results match mla_decode within rounding, not bit for bit.
- * The first call on a device looks up the array's device address; make it before
- * any stream capture.  All calls on a device share the array (it keeps the last
+ * The first call on a device looks up the array's device address
+ * (cudaGetSymbolAddress).  All calls on a device share the array (it keeps the last
  * call's contents; nothing in it must start at zero): calls that overlap on the GPU
  * race and must be serialised by the caller.
  */
@@ -233,10 +232,12 @@ int mla_selected_decode_kernel(int heads);
 
 /*
  * Per-launch device timing.  While enabled, every mla_decode records CUDA events
- * around each of its launches (schedule, decode, combine) on its stream.
- * mla_timing_read synchronises on the last event and writes, for each of the
- * three launches, the summed milliseconds since enabling into ms[0..2], and the
- * number of recorded calls into *calls; it then clears the record.
+ * around each of its launches on its stream.  mla_timing_read synchronises on the
+ * last event and writes the summed milliseconds since enabling into ms[0..2] --
+ * ms[0] the split schedule (no launch of its own: every decode CTA derives its page
+ * range from the lengths, so this is the empty interval between two events), ms[1]
+ * the decode, ms[2] the combine -- and the number of recorded calls into *calls; it
+ * then clears the record.
  */
 mla_status_t mla_timing_enable(int enable);
 mla_status_t mla_timing_read(float ms[3], int* calls);

@@ -332,13 +332,15 @@ mla_status_t decode_call(const void* q, const void* kv_cache, const int32_t* blo
   a.hq = heads / s_q;
   a.row_stride = heads;
   a.row0 = 0;
-  const int min_pages = g_knobs[MLA_KNOB_MIN_PAGES].load() > 0 ? g_knobs[MLA_KNOB_MIN_PAGES].load() : 4;
+  a.min_pages = g_knobs[MLA_KNOB_MIN_PAGES].load() > 0 ? g_knobs[MLA_KNOB_MIN_PAGES].load() : 4;
+  a.granule = decode_granule(kernel);
+  a.whole_slack = schedule_whole_slack();
 
+  // The decode CTAs derive the split schedule themselves: the timing slot of the
+  // schedule (events 0 -> 1) stays empty.
   record_event(*d, 0, stream);
-  cudaError_t e = launch_schedule(cache_seqlens, batch, max_blocks, min_pages, decode_granule(kernel),
-                                  schedule_whole_slack(), a.sched, d->err, stream);
-  if (e != cudaSuccess) return cuda_fail(e, "schedule launch");
   record_event(*d, 1, stream);
+  cudaError_t e = cudaSuccess;
   for (int r0 = 0; r0 < heads; r0 += group) {
     a.row0 = r0;
     a.heads = std::min(group, heads - r0);

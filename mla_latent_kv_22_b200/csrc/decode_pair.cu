@@ -52,6 +52,7 @@
 #include "mla_device.cuh"
 #include "mla_internal.h"
 #include "sm100_ptx.cuh"
+#include "worker_range.cuh"
 
 namespace mla {
 namespace {
@@ -103,17 +104,17 @@ struct Piece {
   int b, pa, pe;
 };
 
-// Iterates the sequence pieces of worker w in schedule order.
+// Iterates the sequence pieces of a worker's range in schedule order.
 struct PieceIter {
-  const Schedule& sc;
   WorkerRange rg;
   int b;
-  __device__ PieceIter(const Schedule& s, int w) : sc(s), rg(s.ranges[w]), b(rg.b0) {}
-  __device__ bool next(Piece& pc) {
+  __device__ explicit PieceIter(const WorkerRange& r) : rg(r), b(r.b0) {}
+  // The lengths are passed at each call, so the iterator holds no copy of them.
+  __device__ bool next(Piece& pc, const int32_t* seqlens, int max_blocks) {
     if (rg.b0 < 0) return false;
     while (b <= rg.b1) {
       const int cur = b++;
-      const int n = sc.seq_start[cur + 1] - sc.seq_start[cur];
+      const int n = seq_pages(seqlens, max_blocks, cur);
       const int pa = (cur == rg.b0) ? rg.p0 : 0;
       const int pe = (cur == rg.b1) ? rg.p1 : n;
       if (pa < pe) {
@@ -200,11 +201,10 @@ struct PieceInfo {
 };
 
 __device__ __forceinline__ PieceInfo piece_info(const DecodeArgs& a, const Piece& pc) {
-  const Schedule& sc = a.sched;
   PieceInfo f;
   f.steps = (pc.pe - pc.pa + kStepPages - 1) / kStepPages;
   const int T = a.seqlens[pc.b];
-  const int nseq = sc.seq_start[pc.b + 1] - sc.seq_start[pc.b];
+  const int nseq = seq_pages(a.seqlens, a.max_blocks, pc.b);
   f.tail_valid = T & (kPage - 1);
   f.tail_pp = (pc.pe == nseq && f.tail_valid != 0) ? pc.pe - 1 : -1;
   return f;
@@ -218,6 +218,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   __shared__ __align__(8) uint64_t bars[kNumBars];
   __shared__ uint32_t tmem_base_s;
   __shared__ int abort_s;
+  __shared__ RangeScratch range_s;
   __shared__ float mx_s[2][2][2][64];  // [step parity][token half][column half][head]
   __shared__ float lsum_s[2][2][64];   // [token half][column half][head]
 
@@ -265,8 +266,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   __syncthreads();
   cluster_sync();  // barriers and tensor memory of both CTAs ready before any remote access
   tc_fence_after();
-  // Everything above overlaps the schedule grid; from here on its output is read.
+  // Everything above overlaps the previous grid on the stream; from here on its writes
+  // (the lengths, q, the block table) are visible.
   grid_dep_wait();
+  // Every thread takes part in deriving this worker's page range (and this CTA's share of
+  // the sequence records the combine reads).
+  derive_worker_range(a.seqlens, a.batch, a.max_blocks, a.sched.num_workers, a.min_pages, a.granule,
+                      a.whole_slack, a.sched.seq, a.err, w, range_s);
+  // Each role reads the range from shared memory where it starts (volatile, so the
+  // read is not hoisted and the range is not held in registers across the kernel).
+  auto rg_load = [&]() {
+    const volatile WorkerRange& v = range_s.rg;
+    return WorkerRange{v.b0, v.p0, v.b1, v.p1};
+  };
   const uint32_t tmem = tmem_base_s;
   Ctl ctl{a.err, &abort_s, map_to_rank(smem_u32(&abort_s), peer), limit_ns};
   // Barriers of CTA 0 as cluster addresses (remote arrivals, completions of the pair's loads).
@@ -275,7 +287,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
-      PieceIter pi(sc, w);
+      PieceIter pi(rg_load());
       Piece pc;
       int k = 0, piece = 0;  // ring fills, pieces
       bool ok = true;
@@ -303,7 +315,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         ++k;
         return true;
       };
-      while (ok && pi.next(pc)) {
+      while (ok && pi.next(pc, a.seqlens, a.max_blocks)) {
         const PieceInfo f = piece_info(a, pc);
         const int b = pc.b;
         // Row y of the piece's page pp (out-of-range page ids and pages past the piece
@@ -380,7 +392,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     // The whole warp runs the issue loop in uniform control flow and one elected lane
     // issues each MMA and commit, so the issue path stays short.
     if (rank == 0) {
-      PieceIter pi(sc, w);
+      PieceIter pi(rg_load());
       Piece pc;
       int g = 0, piece = 0, tails = 0;
       bool ok = true;
@@ -452,7 +464,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         mma_commit_pair_elect(bar(kODone), kBothCtas);
         return true;
       };
-      while (ok && pi.next(pc)) {
+      while (ok && pi.next(pc, a.seqlens, a.max_blocks)) {
         const PieceInfo f = piece_info(a, pc);
         if (!__all_sync(0xffffffffu, wait_bar(bar(kQFull), piece & 1, ctl)) ||
             !__all_sync(0xffffffffu, wait_bar(bar(kQReady), piece & 1, ctl))) {
@@ -480,7 +492,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   } else if (warp == 2) {
     // ------------------------------------------------------------ value rows past a
     // sequence's end, in the value slots of its ragged last page
-    PieceIter pi(sc, w);
+    PieceIter pi(rg_load());
     Piece pc;
     int k = 0;
     int tcnt[kSlots];
@@ -488,7 +500,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     for (int s = 0; s < kSlots; ++s) tcnt[s] = 0;
     bool ok = true;
     const uint32_t tready0 = bar0(kTReady);
-    while (ok && pi.next(pc)) {
+    while (ok && pi.next(pc, a.seqlens, a.max_blocks)) {
       const PieceInfo f = piece_info(a, pc);
       for (int i = 0; i <= f.steps && ok; ++i) {
         if (i < f.steps) k += kQKSlots;
@@ -571,15 +583,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       __syncwarp();
       if (lane == 0) arrive_cta0(rank, bar(kQReady), qready0);
     };
-    PieceIter pi(sc, w), pn(sc, w);  // pn runs one piece ahead
+    PieceIter pi(rg_load()), pn(rg_load());  // pn runs one piece ahead
     Piece pc, nc;
-    bool have_next = pn.next(nc);
+    bool have_next = pn.next(nc, a.seqlens, a.max_blocks);
     if (have_next) stage_q(nc.b);  // the first piece's q' (tensor memory is unused so far)
     int g = 0, piece = 0;
     bool ok = true;
 
-    while (ok && pi.next(pc)) {
-      have_next = pn.next(nc);
+    while (ok && pi.next(pc, a.seqlens, a.max_blocks)) {
+      have_next = pn.next(nc, a.seqlens, a.max_blocks);
       const PieceInfo f = piece_info(a, pc);
       const int b = pc.b;
       const int T = a.seqlens[b];
@@ -718,7 +730,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       const bool none = kCausal && l_row == 0.f;  // a causal row that sees no token of the piece
       const float inv = bad ? NAN : (none ? 0.f : 1.f / l_row);
       const float lse_v = bad ? NAN : (none ? -INFINITY : (m + __log2f(l_row)) * kLn2);
-      const bool complete = pc.pa == 0 && pc.pe == sc.seq_start[b + 1] - sc.seq_start[b];
+      const bool complete = pc.pa == 0 && pc.pe == seq_pages(a.seqlens, a.max_blocks, b);
       float* obase;
       float* lbase;
       if (complete) {
@@ -726,7 +738,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         obase = a.out + rbase * kDLatent;
         lbase = a.lse + rbase;
       } else {
-        const int slot = (b == sc.ranges[w].b0) ? w : P + w;
+        const int slot = (b == pi.rg.b0) ? w : P + w;
         obase = sc.part_o + (size_t)slot * a.heads * kDLatent;
         lbase = sc.part_lse + (size_t)slot * a.heads;
       }

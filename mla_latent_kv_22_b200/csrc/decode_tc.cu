@@ -56,6 +56,7 @@
 #include "mla_device.cuh"
 #include "mla_internal.h"
 #include "sm100_ptx.cuh"
+#include "worker_range.cuh"
 
 namespace mla {
 namespace {
@@ -108,17 +109,17 @@ struct Piece {
   int b, pa, pe;
 };
 
-// Iterates the sequence pieces of worker w in schedule order.
+// Iterates the sequence pieces of a worker's range in schedule order.
 struct PieceIter {
-  const Schedule& sc;
   WorkerRange rg;
   int b;
-  __device__ PieceIter(const Schedule& s, int w) : sc(s), rg(s.ranges[w]), b(rg.b0) {}
-  __device__ bool next(Piece& pc) {
+  __device__ explicit PieceIter(const WorkerRange& r) : rg(r), b(r.b0) {}
+  // The lengths are passed at each call, so the iterator holds no copy of them.
+  __device__ bool next(Piece& pc, const int32_t* seqlens, int max_blocks) {
     if (rg.b0 < 0) return false;
     while (b <= rg.b1) {
       const int cur = b++;
-      const int n = sc.seq_start[cur + 1] - sc.seq_start[cur];
+      const int n = seq_pages(seqlens, max_blocks, cur);
       const int pa = (cur == rg.b0) ? rg.p0 : 0;
       const int pe = (cur == rg.b1) ? rg.p1 : n;
       if (pa < pe) {
@@ -194,6 +195,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   __shared__ __align__(8) uint64_t bars[kNumBars];
   __shared__ uint32_t tmem_base_s;
   __shared__ int abort_s;
+  __shared__ RangeScratch range_s;
 
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
@@ -244,24 +246,35 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   __syncthreads();
   cluster_sync();  // barriers of both CTAs initialised before any remote arrive
   tc_fence_after();
-  // Everything above overlaps the schedule grid; from here on its output is read.
+  // Everything above overlaps the previous grid on the stream; from here on its writes
+  // (the lengths, q, the block table) are visible.
   grid_dep_wait();
+  // Every thread takes part in deriving this worker's page range (and this CTA's share of
+  // the sequence records the combine reads).
+  derive_worker_range(a.seqlens, a.batch, a.max_blocks, a.sched.num_workers, a.min_pages, a.granule,
+                      a.whole_slack, a.sched.seq, a.err, w, range_s);
+  // Each role reads the range from shared memory where it starts (volatile, so the
+  // read is not hoisted and the range is not held in registers across the kernel).
+  auto rg_load = [&]() {
+    const volatile WorkerRange& v = range_s.rg;
+    return WorkerRange{v.b0, v.p0, v.b1, v.p1};
+  };
   const uint32_t tmem = tmem_base_s;
   Ctl ctl{a.err, &abort_s, map_to_rank(smem_u32(&abort_s), peer), limit_ns};
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
-      PieceIter pi(sc, w);
+      PieceIter pi(rg_load());
       Piece pc;
       int it = 0;
       bool ok = true;
       // A second walk over the same pages runs kPrefetch pages ahead and pulls this
       // CTA's part of each page into L2, so the loads into the stage ring (whose
       // depth is bounded by shared memory) see L2 rather than HBM latency.
-      PieceIter pf(sc, w);
+      PieceIter pf(rg_load());
       Piece fc;
-      bool fvalid = pf.next(fc);
+      bool fvalid = pf.next(fc, a.seqlens, a.max_blocks);
       int fp = fvalid ? fc.pa : 0;
       auto prefetch_next = [&]() {
         if (!fvalid) return;
@@ -273,12 +286,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           tma_prefetch_l2_2d(&rope_map, kDLatent + 32 * rank, y);
         }
         if (++fp >= fc.pe) {
-          fvalid = pf.next(fc);
+          fvalid = pf.next(fc, a.seqlens, a.max_blocks);
           fp = fvalid ? fc.pa : 0;
         }
       };
       for (int i = 0; i < kPrefetch; ++i) prefetch_next();
-      while (ok && pi.next(pc)) {
+      while (ok && pi.next(pc, a.seqlens, a.max_blocks)) {
         for (int p = pc.pa; p < pc.pe; ++p, ++it) {
           const int s = it % kStages;
           int pid = page_of(a, pc.b, p);  // table read issued before the wait, off the critical path
@@ -305,7 +318,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      PieceIter pi(sc, w);
+      PieceIter pi(rg_load());
       Piece pc;
       int it = 0, piece = 0;
       bool ok = true;
@@ -350,7 +363,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         return mbar_test(bar(kPFull), g & 1) &&
                mbar_test(bar(kVReady + g % kStages), (g / kStages) & 1);
       };
-      while (ok && pi.next(pc)) {
+      while (ok && pi.next(pc, a.seqlens, a.max_blocks)) {
         if (!wait_bar(bar(kQReady), piece & 1, ctl)) { ok = false; break; }
         const int n = pc.pe - pc.pa, end = it + n;
         int gq = it, gp = it;
@@ -408,11 +421,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------ tail rows of V,
     // and receive buffers handed back to the peer
     const uint32_t peer_free = map_to_rank(bar(kPeerFree), peer);
-    PieceIter pi(sc, w);
+    PieceIter pi(rg_load());
     Piece pc;
     int it = 0;
     bool ok = true;
-    while (ok && pi.next(pc)) {
+    while (ok && pi.next(pc, a.seqlens, a.max_blocks)) {
       const int T = a.seqlens[pc.b];
       for (int p = pc.pa; p < pc.pe; ++p, ++it) {
         const int s = it % kStages;
@@ -451,11 +464,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       const uint32_t rx_peer = map_to_rank(s_rx, peer);
       const uint32_t peer_rx_full = map_to_rank(bar(kRxFull), peer);
       mbar_arrive(bar(kTxWritable));  // the send buffer starts free
-      PieceIter pi(sc, w);
+      PieceIter pi(rg_load());
       Piece pc;
       int it = 0;
       bool ok = true;
-      while (ok && pi.next(pc)) {
+      while (ok && pi.next(pc, a.seqlens, a.max_blocks)) {
         for (int p = pc.pa; p < pc.pe; ++p, ++it) {
           // All 8 softmax warps wrote their rows, and the peer has read page it-2 out of
           // its receive buffer u and re-armed it (both buffers start armed).
@@ -499,7 +512,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     const float thr_raw = scale2 > 0.f ? kRescaleThreshold / scale2 : INFINITY;
     uint8_t* txrow = smem + kSmemTx + row * kXRow;
     const int sw2 = (row >> 1) & 3;  // chunk swizzle of 192-byte rows: XOR keeps groups of 4 chunks
-    PieceIter pi(sc, w);
+    PieceIter pi(rg_load());
     Piece pc;
     int it = 0, piece = 0;
     bool ok = true;
@@ -543,7 +556,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       return true;
     };
 
-    while (ok && pi.next(pc)) {
+    while (ok && pi.next(pc, a.seqlens, a.max_blocks)) {
       const int b = pc.b, n = pc.pe - pc.pa;
       const int T = a.seqlens[b];
       // Tokens this row attends to: all T, or its query token's causal window.
@@ -721,7 +734,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       const bool none = kCausal && l_row == 0.f;
       const float inv = bad ? NAN : (none ? 0.f : 1.f / l_row);
       const float lse_v = bad ? NAN : (none ? -INFINITY : (m * scale2 + __log2f(l_row)) * kLn2);
-      const bool complete = pc.pa == 0 && pc.pe == sc.seq_start[b + 1] - sc.seq_start[b];
+      const bool complete = pc.pa == 0 && pc.pe == seq_pages(a.seqlens, a.max_blocks, b);
       float* obase;
       float* lbase;
       if (complete) {
@@ -729,7 +742,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         obase = a.out + rbase * kDLatent;
         lbase = a.lse + rbase;
       } else {
-        const int slot = (b == sc.ranges[w].b0) ? w : P + w;
+        const int slot = (b == pi.rg.b0) ? w : P + w;
         obase = sc.part_o + (size_t)slot * a.heads * kDLatent;
         lbase = sc.part_lse + (size_t)slot * a.heads;
       }

@@ -12,17 +12,17 @@
 
 namespace mla {
 
-// Split schedule, written on the device by the schedule kernel.
+// Split schedule, derived on the device by every decode CTA (worker_range.cuh).
 //
 // The pages of all sequences are laid end to end (sequence-major); worker w takes
 // the contiguous range [w*q, min((w+1)*q, N)) of that list, q = max(ceil(N/P),
-// min_pages).  A worker's range covers a tail of its first sequence, whole middle
-// sequences and a head of its last one.  A sequence that one worker covers
-// entirely is written straight to out/lse; otherwise every worker writes its piece
-// (normalised partial output and its lse) to a partial slot -- slot w when the
-// sequence is the worker's first, slot P + w otherwise -- and the combine kernel
-// merges the pieces by their lse.  Everything depends only on the sequence lengths,
-// the batch size and P.
+// min_pages) rounded up to the kernel's page granule.  A worker's range covers a tail
+// of its first sequence, whole middle sequences and a head of its last one.  A
+// sequence that one worker covers entirely is written straight to out/lse; otherwise
+// every worker writes its piece (normalised partial output and its lse) to a partial
+// slot -- slot w when the sequence is the worker's first, slot P + w otherwise -- and
+// the combine kernel merges the pieces by their lse.  Everything depends only on the
+// sequence lengths, the batch size and P.
 struct WorkerRange {
   int b0, p0;  // first sequence and its first page
   int b1, p1;  // last sequence and one past its last page (b0 < 0: no work)
@@ -35,10 +35,7 @@ struct SeqInfo {
 };
 
 struct Schedule {
-  WorkerRange* ranges;  // [P]
-  int* seq_start;       // [B + 1] prefix sums of pages per sequence
-  SeqInfo* seq;         // [B]
-  int* quota;           // [1] pages per worker q
+  SeqInfo* seq;         // [B], written by the decode grid, read by the combine grid
   float* part_lse;      // [2P, H]  (natural-log lse of each piece)
   float* part_o;        // [2P, H, 512] normalised partial outputs
   int num_workers;      // P
@@ -65,14 +62,12 @@ struct DecodeArgs {
   // sees the first T - s_q + 1 + i cached tokens), of which one launch handles the
   // `heads` rows starting at row0.  s_q = 1, hq = row_stride = heads, row0 = 0 otherwise.
   int s_q, hq, row_stride, row0;
+  // Split schedule, derived by every decode CTA (worker_range.cuh): the least pages per
+  // worker, the page granule of the kernel's steps, and the whole-sequence slack (< 0:
+  // always split).
+  int min_pages, granule, whole_slack;
 };
 
-// granule: the pages per worker are rounded up to a multiple of it (the pair kernel
-// walks its range in steps of 4 pages).  whole_slack >= 0: one whole sequence per worker
-// when batch <= workers and the longest sequence exceeds the split quota by at most
-// whole_slack pages; < 0: always split.
-cudaError_t launch_schedule(const int32_t* seqlens, int batch, int max_blocks, int min_pages, int granule,
-                            int whole_slack, const Schedule& s, int* err, cudaStream_t stream);
 // The whole-sequence slack for the current knobs (a forced worker count always splits).
 int schedule_whole_slack();
 cudaError_t launch_combine(const DecodeArgs& a, cudaStream_t stream);

@@ -1,27 +1,25 @@
 // mla_decode_noalloc: the same decode as mla_decode, for callers that must not
 // allocate device memory.
 //
-// mla_decode keeps its split partials and schedule in a workspace that it grows
-// with cudaMalloc on first need (or that the caller hands over).  Some callers can
-// do neither: a serving runtime that has already reserved all device memory for
-// its own pool, code that runs while a stream is being captured into a CUDA graph
-// (cudaMalloc is not capturable), or latency-critical paths where cudaMalloc's
-// implicit device synchronisation is not acceptable.  This variant takes its
+// mla_decode keeps its split partials and per-sequence records in a workspace that
+// it grows with cudaMalloc on first need (or that the caller hands over).  Some
+// callers can do neither: a serving runtime that has already reserved all device
+// memory for its own pool, or latency-critical paths where cudaMalloc's implicit
+// device synchronisation is not acceptable.  This variant takes its
 // scratch from one file-scope __device__ array instead: kNoAllocScratchBytes
 // (32 MiB) that every GPU which loads the library holds until the process exits.
 //
 // Contract:
-//  - Sizes whose schedule and partials do not fit the array are rejected with
+//  - Sizes whose records and partials do not fit the array are rejected with
 //    MLA_ERR_UNSUPPORTED before anything is launched.  To fit, the call may use
 //    fewer split workers than mla_decode (at 128 heads at most 63 CTA pairs), so
 //    its results agree with mla_decode's within rounding, not bit for bit.
 //  - The first call on a device looks up the array's device address
-//    (cudaGetSymbolAddress, with that device current); make that first call
-//    before any stream capture.
+//    (cudaGetSymbolAddress, with that device current).
 //  - Every call on a device shares the one array, and the array keeps the last
-//    call's contents.  Nothing in it has to start at zero: each call rewrites the
-//    schedule before the decode reads it and writes every partial slot before the
-//    combine reads it.  Calls that overlap on the GPU (other streams, other host
+//    call's contents.  Nothing in it has to start at zero: the decode grid of each call
+//    rewrites the per-sequence records and every partial slot before the combine
+//    reads them.  Calls that overlap on the GPU (other streams, other host
 //    threads) race on the array and must be serialised by the caller.
 //  - No cudaMalloc, cudaFree or allocating library call is made.
 #include <cuda_runtime.h>
@@ -120,11 +118,10 @@ extern "C" mla_status_t mla_decode_noalloc(const void* q, const void* kv_cache, 
   a.row_stride = heads;
   a.row0 = 0;
   const int mp = mla::knob_value(MLA_KNOB_MIN_PAGES);
-  const int min_pages = mp > 0 ? mp : 4;
+  a.min_pages = mp > 0 ? mp : 4;
+  a.granule = mla::decode_granule(kernel);
+  a.whole_slack = mla::schedule_whole_slack();
 
-  e = mla::launch_schedule(cache_seqlens, batch, max_blocks, min_pages, mla::decode_granule(kernel),
-                           mla::schedule_whole_slack(), a.sched, err, stream);
-  if (e != cudaSuccess) return reject(MLA_ERR_CUDA, "schedule launch failed");
   e = mla::launch_decode(kernel, a, stream);
   if (e != cudaSuccess) return reject(MLA_ERR_CUDA, "decode launch failed");
   e = mla::launch_combine(a, stream);

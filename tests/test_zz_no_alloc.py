@@ -1,6 +1,6 @@
 """mla_decode_noalloc: the decode for callers that cannot allocate device memory
-(a runtime that has reserved all device memory for its own pool, code running
-under stream capture, paths that cannot absorb cudaMalloc's device sync).  It uses
+(a runtime that has reserved all device memory for its own pool, paths that cannot
+absorb cudaMalloc's device sync).  It uses
 the library's static device scratch instead of the workspace.
 
 Checked through the C ABI against the fp64 oracle (mla_decode_ref) and against
