@@ -742,18 +742,34 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         obase = sc.part_o + (size_t)slot * a.heads * kDLatent;
         lbase = sc.part_lse + (size_t)slot * a.heads;
       }
+      // The warp's 32 rows x 128 dims leave through its own 4 KB of the P buffer (free:
+      // every value MMA of the piece is done, and this warp writes the next piece's P
+      // there only after this loop), 32 dims at a time: each thread stages its row (16-byte
+      // chunks XOR-swizzled by row, so neither side conflicts on banks), then 8 lanes store
+      // one row's 128 contiguous bytes -- against 32 rows touched by every store when each
+      // thread wrote its own row.
+      uint8_t* const stage = smem + kOffP + (2 * hh + c) * kBox + 32 * (q & 1) * 128;
+      const int sr = lane >> 3, sk = lane & 7;  // staged row within a group of 4, chunk
 #pragma unroll 1
       for (int cc = 0; cc < 4; ++cc) {
         uint32_t r[32];
         tmem_ld32(tmem + lane_addr + kColO + 128 * c + 32 * cc, r);
         tmem_wait_ld();
-        if (row < a.heads) {
-          float4* dst = reinterpret_cast<float4*>(obase + (size_t)row * kDLatent + 256 * c + 128 * hh + 32 * cc);
 #pragma unroll
-          for (int e = 0; e < 8; ++e)
-            dst[e] = make_float4(__uint_as_float(r[4 * e]) * inv, __uint_as_float(r[4 * e + 1]) * inv,
-                                 __uint_as_float(r[4 * e + 2]) * inv, __uint_as_float(r[4 * e + 3]) * inv);
+        for (int e = 0; e < 8; ++e)
+          *reinterpret_cast<float4*>(stage + lane * 128 + ((e ^ (lane & 7)) * 16)) =
+              make_float4(__uint_as_float(r[4 * e]) * inv, __uint_as_float(r[4 * e + 1]) * inv,
+                          __uint_as_float(r[4 * e + 2]) * inv, __uint_as_float(r[4 * e + 3]) * inv);
+        __syncwarp();
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const int rr = 4 * i + sr;                            // staged row = lane rr of this warp
+          const int orow = 64 * (int)rank + 32 * (q & 1) + rr;  // its row of the launch
+          const float4 v = *reinterpret_cast<const float4*>(stage + rr * 128 + ((sk ^ (rr & 7)) * 16));
+          if (orow < a.heads)
+            *reinterpret_cast<float4*>(obase + (size_t)orow * kDLatent + 256 * c + 128 * hh + 32 * cc + 4 * sk) = v;
         }
+        __syncwarp();  // the staging area is rewritten by the next 32 dims
       }
       if (hh == 0 && c == 0 && row < a.heads) lbase[row] = lse_v;
       tc_fence_before();
