@@ -44,16 +44,14 @@ def _replay_matches_eager(run, inputs_a, inputs_b, outs):
     del g
 
 
-@pytest.mark.parametrize("entry", ["mla_decode", "mla_decode_noalloc"])
-def test_decode_replayed_from_a_graph(entry):
+def test_decode_replayed_from_a_graph():
     a = S.make_decode_case(4, 128, [100, 700, 64, 1], seed=91, poison=True)
     b = S.make_decode_case(4, 128, [100, 700, 64, 1], seed=92, poison=True)
     q, kv, bt, sl = upload(a)
     q_b = bf16_dev(b.q)
     out = torch.empty(4, 128, 512, device="cuda")
     lse = torch.empty(4, 128, device="cuda")
-    fn = getattr(M, entry)
-    _replay_matches_eager(lambda: fn(q, kv, bt, sl, out, lse, a.softmax_scale),
+    _replay_matches_eager(lambda: M.mla_decode(q, kv, bt, sl, out, lse, a.softmax_scale),
                           [(q, bf16_dev(a.q))], [(q, q_b)], [out, lse])
 
 
