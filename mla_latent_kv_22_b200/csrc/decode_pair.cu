@@ -73,9 +73,19 @@ constexpr int kOffP = kQSmemBoxes * kBox;
 constexpr int kOffRing = kOffP + 4 * kBox;
 constexpr int kSmemBytes = kOffRing + kSlots * kSlotBytes;  // 204800
 constexpr int kSmemAlloc = kSmemBytes + 1024;               // + alignment slack
+// Every region lies inside the allocation, and the allocation, with the kernel's static
+// shared memory (under 4 KB), inside the 227 KB a CTA may have.
+static_assert(kOffQ + kQSmemBoxes * kBox <= kOffP && kOffP + 4 * kBox <= kOffRing &&
+                  kOffRing + kSlots * kSlotBytes <= kSmemBytes,
+              "shared-memory regions overlap or leave the allocation");
+static_assert(kSmemAlloc + 4096 <= 232448, "dynamic + static shared memory above the per-CTA limit");
+static_assert(kOffP % 1024 == 0 && kOffRing % 1024 == 0 && kSlotBytes % 1024 == 0 && kBox % 1024 == 0,
+              "128B-swizzled tiles must start on 1024-byte boundaries");
 
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColO = 0, kColS = 256, kColQ = 384;
+static_assert(kColO + 256 <= kColS && kColS + 128 <= kColQ && kColQ + 2 * kQTmemBoxes * 16 <= kTmemCols,
+              "tensor-memory regions overlap or leave the allocation");
 constexpr uint32_t kIdescQK = idesc_bf16_f32(128, 256, 0, 0);  // A q' K-major, B rows K-major
 constexpr uint32_t kIdescPV = idesc_bf16_f32(128, 256, 0, 1);  // A P K-major, B rows MN-major
 constexpr uint16_t kBothCtas = 3;

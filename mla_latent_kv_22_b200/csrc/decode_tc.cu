@@ -74,11 +74,19 @@ constexpr int kSmemTx = kStages * kStageBytes;                // 147456: send bu
 constexpr int kSmemRx = kSmemTx + kXBytes;                    // 172032: 2 receive buffers
 constexpr int kSmemBytes = kSmemRx + 2 * kXBytes;             // 221184
 constexpr int kSmemAlloc = kSmemBytes + 1024;                 // + alignment slack
+// Every region lies inside the allocation, and the allocation, with the kernel's static
+// shared memory (under 4 KB), inside the 227 KB a CTA may have.
+static_assert(kStages * kStageBytes <= kSmemTx && kSmemTx + kXBytes <= kSmemRx && kSmemRx + 2 * kXBytes <= kSmemBytes,
+              "shared-memory regions overlap or leave the allocation");
+static_assert(kSmemAlloc + 4096 <= 232448, "dynamic + static shared memory above the per-CTA limit");
+static_assert(kStageBytes % 1024 == 0, "swizzled stage tiles must start on 1024-byte boundaries");
 
 constexpr uint32_t kTmemCols = 512;
 // O fp32 [0,256); q' (latent 256 dims, then this CTA's 32 rope dims) as bf16 pairs
 // [256,400); S fp32 [400,464); P bf16 pairs [464,496).
 constexpr uint32_t kColO = 0, kColQ = 256, kColS = 400, kColP = 464;
+static_assert(kColO + 256 <= kColQ && kColQ + 144 <= kColS && kColS + 64 <= kColP && kColP + 32 <= kTmemCols,
+              "tensor-memory regions overlap or leave the allocation");
 
 constexpr uint32_t kIdescQK = idesc_bf16_f32(128, 64, 0, 0);   // A (q', TMEM), B K-major
 constexpr uint32_t kIdescPV = idesc_bf16_f32(128, 256, 0, 1);  // A (P, TMEM), B MN-major
