@@ -56,28 +56,50 @@ def algorithmic_flops(b: int, h: int, t: int) -> int:
     return 2 * b * h * t * (D + DV)
 
 
-def split_partial_bytes(seqlens, heads: int, workers: int, min_pages: int = 4, granule: int = 4,
-                        whole_slack: int = 16) -> int:
+def split_pieces(seqlens, workers: int, min_pages: int = 4, granule: int = 4, whole_slack: int = 16,
+                 piece_cost: int = 8):
+    """The library's split rule for the default knobs, restated on the host: per worker, its
+    pieces as (sequence, first page, end page).  Sequences are laid end to end, each as
+    piece_cost units of fixed cost followed by its pages; worker w takes the pages inside
+    units [w q, (w+1) q), q = max(ceil(units / P), min_pages) rounded up to the granule.
+    When batch <= P and the longest sequence is at most whole_slack pages above the
+    pages-only share, every sequence runs whole on worker b."""
+    pages = [(int(t) + PAGE - 1) // PAGE if 0 <= int(t) else 0 for t in seqlens]
+    b_n = len(pages)
+
+    def share(total):
+        q = max(-(-total // workers), min_pages, 1)
+        return -(-q // granule) * granule
+
+    if whole_slack >= 0 and b_n <= workers and max(pages, default=0) <= share(sum(pages)) + whole_slack:
+        return [[(b, 0, n)] if n > 0 else [] for b, n in enumerate(pages)]
+    units = [n + piece_cost if n > 0 else 0 for n in pages]
+    total = sum(units)
+    q = share(total)
+    starts = [0]
+    for u in units:
+        starts.append(starts[-1] + u)
+    plan = []
+    for w in range(-(-total // q)):
+        g0, g1 = w * q, min(w * q + q, total)
+        pieces = []
+        for b, n in enumerate(pages):
+            pos = starts[b] + piece_cost
+            lo, hi = max(g0, pos), min(g1, pos + n)
+            if n > 0 and lo < hi:
+                pieces.append((b, lo - pos, hi - pos))
+        plan.append(pieces)
+    return plan
+
+
+def split_partial_bytes(seqlens, heads: int, workers: int) -> int:
     """Bytes of split partials one decode step moves: every piece of a split sequence
     writes its normalised output (512 fp32 per head) and lse, and the combine reads them
-    back.  The split follows the library's schedule rule for the default knobs (pages
-    laid end to end, q = max(ceil(N / P), min_pages) rounded up to the granule; one
-    whole sequence per worker when batch <= P and the longest sequence is at most
-    whole_slack pages above q)."""
+    back (the split as `split_pieces` gives it)."""
     pages = [(int(t) + PAGE - 1) // PAGE for t in seqlens]
-    n_all, b = sum(pages), len(pages)
-    q = max(-(-n_all // workers), min_pages, 1)
-    q = -(-q // granule) * granule
-    if b <= workers and max(pages) <= q + whole_slack:
-        return 0
-    pieces, st = 0, 0
-    for n in pages:
-        if n > 0:
-            k = (st + n - 1) // q - st // q + 1
-            if k > 1:
-                pieces += k
-        st += n
-    return 2 * pieces * heads * (DV + 1) * 4
+    split = sum(1 for pieces in split_pieces(seqlens, workers) for (b, lo, hi) in pieces
+                if not (lo == 0 and hi == pages[b]))
+    return 2 * split * heads * (DV + 1) * 4
 
 
 def measured_peaks() -> tuple[dict, str]:

@@ -218,11 +218,17 @@ typedef enum {
   MLA_KNOB_WAIT_LIMIT = 3,      /* > 0: time limit of bounded device waits in ms; 0 = 2000  */
   MLA_KNOB_WITHHOLD_ARRIVE = 4, /* 1: the decode kernel's producer skips one load, so the
                                    consumer's bounded wait must run out (timeout test)      */
-  MLA_KNOB_SPLIT_POLICY = 5     /* 0 = auto: one whole sequence per worker when batch <= the
+  MLA_KNOB_SPLIT_POLICY = 5,    /* 0 = auto: one whole sequence per worker when batch <= the
                                    worker count and the longest sequence is at most 16 pages
                                    above the split quota, else split; 1 = always split;
                                    2 = whole sequences whenever batch <= the worker count.
                                    A forced MLA_KNOB_NUM_WORKERS always splits.             */
+  MLA_KNOB_PIECE_COST = 6       /* pages a split charges each sequence for its fixed cost
+                                   (q' staging, pipeline fill, epilogue) when it lays the
+                                   sequences end to end and cuts equal shares: 0 = auto (8,
+                                   a multiple of the 4-page step, so pieces of step-aligned
+                                   sequences stay aligned); k > 0: k - 1 pages (1 = split
+                                   by pages alone)                                          */
 } mla_knob_t;
 mla_status_t mla_set_knob(mla_knob_t knob, int value);
 int mla_get_knob(mla_knob_t knob);

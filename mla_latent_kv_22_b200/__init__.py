@@ -27,7 +27,8 @@ STATUS = {
     0: "MLA_OK", 1: "MLA_ERR_INVALID_ARG", 2: "MLA_ERR_UNSUPPORTED", 3: "MLA_ERR_WORKSPACE", 4: "MLA_ERR_CUDA",
     5: "MLA_ERR_DEVICE_BAD_PAGE", 6: "MLA_ERR_DEVICE_TIMEOUT",
 }
-KNOB = {"num_workers": 0, "min_pages": 1, "decode_kernel": 2, "wait_limit": 3, "withhold_arrive": 4, "split_policy": 5}
+KNOB = {"num_workers": 0, "min_pages": 1, "decode_kernel": 2, "wait_limit": 3, "withhold_arrive": 4, "split_policy": 5,
+        "piece_cost": 6}
 
 D_LATENT, D_ROPE, D_QK, PAGE, D_NOPE, D_V, MAX_HEADS = 512, 64, 576, 64, 128, 128, 128
 

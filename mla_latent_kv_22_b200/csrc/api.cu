@@ -157,6 +157,11 @@ int schedule_whole_slack() {
   return v == 0 ? 16 : v == 1 ? -1 : 1 << 30;
 }
 
+int schedule_piece_cost() {
+  const int v = g_knobs[MLA_KNOB_PIECE_COST].load();
+  return v > 0 ? v - 1 : 8;
+}
+
 PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
   static std::once_flag once;
@@ -335,6 +340,7 @@ mla_status_t decode_call(const void* q, const void* kv_cache, const int32_t* blo
   a.min_pages = g_knobs[MLA_KNOB_MIN_PAGES].load() > 0 ? g_knobs[MLA_KNOB_MIN_PAGES].load() : 4;
   a.granule = decode_granule(kernel);
   a.whole_slack = schedule_whole_slack();
+  a.piece_cost = schedule_piece_cost();
 
   // The decode CTAs derive the split schedule themselves: the timing slot of the
   // schedule (events 0 -> 1) stays empty.

@@ -260,7 +260,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   // Every thread takes part in deriving this worker's page range (and this CTA's share of
   // the sequence records the combine reads).
   derive_worker_range(a.seqlens, a.batch, a.max_blocks, a.sched.num_workers, a.min_pages, a.granule,
-                      a.whole_slack, a.sched.seq, a.err, w, range_s);
+                      a.whole_slack, a.piece_cost, a.sched.seq, a.err, w, range_s);
   // Each role reads the range from shared memory where it starts (volatile, so the
   // read is not hoisted and the range is not held in registers across the kernel).
   auto rg_load = [&]() {

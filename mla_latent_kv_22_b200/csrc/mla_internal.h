@@ -63,13 +63,15 @@ struct DecodeArgs {
   // `heads` rows starting at row0.  s_q = 1, hq = row_stride = heads, row0 = 0 otherwise.
   int s_q, hq, row_stride, row0;
   // Split schedule, derived by every decode CTA (worker_range.cuh): the least pages per
-  // worker, the page granule of the kernel's steps, and the whole-sequence slack (< 0:
-  // always split).
-  int min_pages, granule, whole_slack;
+  // worker, the page granule of the kernel's steps, the whole-sequence slack (< 0:
+  // always split), and the pages a piece is charged for its fixed cost.
+  int min_pages, granule, whole_slack, piece_cost;
 };
 
 // The whole-sequence slack for the current knobs (a forced worker count always splits).
 int schedule_whole_slack();
+// The pages a split charges each sequence for its fixed cost, for the current knobs.
+int schedule_piece_cost();
 cudaError_t launch_combine(const DecodeArgs& a, cudaStream_t stream);
 cudaError_t launch_absorb_q(const __nv_bfloat16* q_nope, const __nv_bfloat16* q_rope,
                             const __nv_bfloat16* w_uk, __nv_bfloat16* q_out, int batch, int heads, int* err,

@@ -121,6 +121,7 @@ extern "C" mla_status_t mla_decode_noalloc(const void* q, const void* kv_cache, 
   a.min_pages = mp > 0 ? mp : 4;
   a.granule = mla::decode_granule(kernel);
   a.whole_slack = mla::schedule_whole_slack();
+  a.piece_cost = mla::schedule_piece_cost();
 
   e = mla::launch_decode(kernel, a, stream);
   if (e != cudaSuccess) return reject(MLA_ERR_CUDA, "decode launch failed");
