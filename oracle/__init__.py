@@ -40,3 +40,4 @@ from .mla_oracle import (  # noqa: F401
     cache_elements_per_token,
     latent_cache_bytes,
 )
+from .fp8_cache import e4m3_to_f64, dequant_rows, mla_decode_fp8_ref  # noqa: F401

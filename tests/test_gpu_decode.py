@@ -31,7 +31,8 @@ def kernel(request):
     split by heads (pair-wide MMAs)."""
     M.mla_set_knob("decode_kernel", request.param)
     yield request.param
-    for k in ("num_workers", "min_pages", "decode_kernel", "wait_limit", "withhold_arrive", "split_policy"):
+    for k in ("num_workers", "min_pages", "decode_kernel", "wait_limit", "withhold_arrive", "split_policy",
+              "piece_cost"):
         M.mla_set_knob(k, 0)
 
 
@@ -54,6 +55,17 @@ def test_config3_varlen_full():
     out, lse, err = run_decode(case)
     assert err == 0
     assert_close(out, lse, *oracle_for(case), "config 3 var-len")
+
+
+@pytest.mark.parametrize("piece_cost", [1, 4, 13, 41])
+def test_split_piece_cost_keeps_parity(piece_cost):
+    """The split charges each sequence (knob - 1) pages of fixed cost: every charge moves the
+    cut points (pieces of 1 to 3 per worker, some workers with none), never the result."""
+    M.mla_set_knob("piece_cost", piece_cost)
+    case = S.make_decode_case(24, 128, S.uniform_seqlens(41, 24, 1, 3000), seed=41, poison=True)
+    out, lse, err = run_decode(case)
+    assert err == 0
+    assert_close(out, lse, *oracle_for(case), f"piece cost {piece_cost - 1}")
 
 
 def test_config3_headline_sampled():
