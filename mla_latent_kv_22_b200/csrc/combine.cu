@@ -18,7 +18,7 @@ namespace {
 constexpr int kWarps = 4;
 
 __global__ void __launch_bounds__(kWarps * 32) combine_kernel(DecodeArgs a) {
-  grid_dep_launch_dependents();  // the next grid (absorb_o, or the next call's schedule) may launch; it waits for this one
+  grid_dep_launch_dependents();  // the next grid (absorb_o, or the next call's decode) may launch; it waits for this one
   grid_dep_wait();  // the decode grid's partials are complete and visible
   const int b = blockIdx.x;
   const int lane = threadIdx.x & 31;

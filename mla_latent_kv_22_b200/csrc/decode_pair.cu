@@ -856,8 +856,9 @@ cudaError_t launch_decode_pair(const DecodeArgs& a, cudaStream_t stream) {
       return cudaErrorInvalidValue;
   }
   const uint64_t limit_ns = (uint64_t)(a.wait_limit > 0 ? a.wait_limit : 1000) * 1000000ull;  // wait_limit in ms
-  // Launched as a programmatic dependent of the schedule grid: the prologue (barrier
-  // set-up, tensor-memory allocation, descriptor prefetch) overlaps it.
+  // Launched as a programmatic dependent of whatever precedes it on the stream (the
+  // previous call's combine, or the grid that wrote q'): the prologue (barrier set-up,
+  // tensor-memory allocation, descriptor prefetch) overlaps that grid's tail.
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2 * a.sched.num_workers, 1, 1);
   cfg.blockDim = dim3(kThreads, 1, 1);

@@ -832,8 +832,9 @@ cudaError_t launch_decode_tc(const DecodeArgs& a, cudaStream_t stream) {
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
   const uint64_t limit_ns = (uint64_t)(a.wait_limit > 0 ? a.wait_limit : 1000) * 1000000ull;  // wait_limit in ms
-  // Launched as a programmatic dependent of the schedule grid: the prologue (barrier
-  // set-up, TMEM allocation, descriptor prefetch) overlaps it.
+  // Launched as a programmatic dependent of whatever precedes it on the stream (the
+  // previous call's combine, or the grid that wrote q'): the prologue (barrier set-up,
+  // TMEM allocation, descriptor prefetch) overlaps that grid's tail.
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2 * a.sched.num_workers, 1, 1);
   cfg.blockDim = dim3(kThreads, 1, 1);
