@@ -227,8 +227,8 @@ typedef enum {
                                    (q' staging, pipeline fill, epilogue) when it lays the
                                    sequences end to end and cuts equal shares: 0 = auto (8,
                                    a multiple of the 4-page step, so pieces of step-aligned
-                                   sequences stay aligned); k > 0: k - 1 pages (1 = split
-                                   by pages alone)                                          */
+                                   sequences stay aligned); k > 0: min(k - 1, 256) pages 
+                                   (1 = split by pages alone)                               */
 } mla_knob_t;
 mla_status_t mla_set_knob(mla_knob_t knob, int value);
 int mla_get_knob(mla_knob_t knob);

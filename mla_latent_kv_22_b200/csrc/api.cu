@@ -159,7 +159,7 @@ int schedule_whole_slack() {
 
 int schedule_piece_cost() {
   const int v = g_knobs[MLA_KNOB_PIECE_COST].load();
-  return v > 0 ? v - 1 : 8;
+  return v > 0 ? std::min(v - 1, kMaxPieceCost) : 8;
 }
 
 PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
@@ -298,6 +298,8 @@ mla_status_t decode_call(const void* q, const void* kv_cache, const int32_t* blo
   if (block_table && num_pages < 1) return fail(MLA_ERR_INVALID_ARG, "paged cache with num_pages < 1");
   if ((long long)batch * max_blocks > (1LL << 31) - 1 || (long long)max_blocks * MLA_PAGE_TOKENS > (1LL << 30))
     return fail(MLA_ERR_UNSUPPORTED, "cache too large for 32-bit page indexing");
+  if ((long long)batch * ((long long)max_blocks + kMaxPieceCost) > (1LL << 31) - 1)
+    return fail(MLA_ERR_UNSUPPORTED, "batch too large for the 32-bit split schedule");
   if (!aligned16(q) || !aligned16(kv_cache) || !aligned16(out))
     return fail(MLA_ERR_INVALID_ARG, "q, kv_cache and out must be 16-byte aligned");
   if ((reinterpret_cast<uintptr_t>(block_table) & 3u) || (reinterpret_cast<uintptr_t>(cache_seqlens) & 3u) ||

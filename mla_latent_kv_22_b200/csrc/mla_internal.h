@@ -70,7 +70,10 @@ struct DecodeArgs {
 
 // The whole-sequence slack for the current knobs (a forced worker count always splits).
 int schedule_whole_slack();
-// The pages a split charges each sequence for its fixed cost, for the current knobs.
+// The pages a split charges each sequence for its fixed cost, for the current knobs (at
+// most kMaxPieceCost, so that batch x (max_blocks + cost) units fit the device's 32-bit
+// schedule arithmetic whenever the host's size check passes).
+constexpr int kMaxPieceCost = 256;
 int schedule_piece_cost();
 cudaError_t launch_combine(const DecodeArgs& a, cudaStream_t stream);
 cudaError_t launch_absorb_q(const __nv_bfloat16* q_nope, const __nv_bfloat16* q_rope,

@@ -60,6 +60,8 @@ extern "C" mla_status_t mla_decode_noalloc(const void* q, const void* kv_cache, 
   if (block_table && num_pages < 1) return reject(MLA_ERR_INVALID_ARG, "paged cache with num_pages < 1");
   if ((long long)batch * max_blocks > (1LL << 31) - 1 || (long long)max_blocks * MLA_PAGE_TOKENS > (1LL << 30))
     return reject(MLA_ERR_UNSUPPORTED, "cache too large for 32-bit page indexing");
+  if ((long long)batch * ((long long)max_blocks + mla::kMaxPieceCost) > (1LL << 31) - 1)
+    return reject(MLA_ERR_UNSUPPORTED, "batch too large for the 32-bit split schedule");
   if (!aligned16(q) || !aligned16(kv_cache) || !aligned16(out))
     return reject(MLA_ERR_INVALID_ARG, "q, kv_cache and out must be 16-byte aligned");
   if ((reinterpret_cast<uintptr_t>(block_table) & 3u) || (reinterpret_cast<uintptr_t>(cache_seqlens) & 3u) ||

@@ -50,6 +50,8 @@ def _decode(**kw):
     (dict(q=24), 1), (dict(kv=8), 1), (dict(out=4), 1), (dict(lse=2), 1),
     (dict(bt=16, num_pages=0), 1), (dict(scale=float("nan")), 1), (dict(scale=float("inf")), 1),
     (dict(max_blocks=1 << 25), 2),
+    # batch x (table width + the largest piece cost) must fit the device's 32-bit split arithmetic
+    (dict(B=8_000_000, max_blocks=16), 2),
 ])
 def test_decode_host_validation(kw, status):
     assert _decode(**kw) == status
@@ -63,6 +65,12 @@ def test_decode_host_validation(kw, status):
 def test_decode_multi_host_validation(s_q, H, q, status):
     assert M.lib.mla_decode_multi(q, 16, None, 16, 16, 16, 2, s_q, H, 10, 4, 0.1, None) == status
     assert M.lib.mla_last_error_message()
+
+
+def test_split_schedule_size_limit_message():
+    assert _decode(B=8_000_000, max_blocks=16) == 2
+    assert b"32-bit split schedule" in M.lib.mla_last_error_message()
+    assert _decode(B=8_000_000, max_blocks=1, q=24) == 1  # 8M x 257 units fit: the next check runs
 
 
 def test_empty_batch_is_a_no_op():
